@@ -1,0 +1,172 @@
+"""ctypes front end of the CoSA CPU oracle (test infrastructure only).
+
+Only tests/, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg
+import this package.  The product path (``block_sparse_attention_kap_b200``)
+never imports, calls or links it.
+
+Every function takes host torch tensors (bf16 inputs as produced by
+``synth``) and returns host tensors.  Semantics: see cosa_oracle.c; each
+step cites the CoSA technical summary (Sec. 2.1-2.3).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+from . import build as _build
+
+_LIB = None
+
+
+class OrShape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in
+                ("B", "Hq", "Hkv", "Nq", "Nkv", "d", "bq", "bk", "s", "paged", "num_pages")]
+
+
+def lib():
+    global _LIB
+    if _LIB is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        P, I, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
+        S = ctypes.POINTER(OrShape)
+        L.oracle_kap.argtypes = [S, P, P, P, D, P, I, I, P, P, P, P, P, I]
+        L.oracle_osk.argtypes = [S, P, P, P, P, P, I, P, P, I, D, P, P, P, I]
+        L.oracle_dense.argtypes = [S, P, P, P, P, P, I, P, P, I, P, P, I]
+        L.oracle_kmax.argtypes = [S, D]
+        L.oracle_causal_blocks.argtypes = [S, I]
+        L.oracle_budget_blocks.argtypes = [I, D]
+        L.oracle_skip_threshold.argtypes = [D, I]
+        L.oracle_skip_threshold.restype = ctypes.c_float
+        L.oracle_pool.argtypes = [P, I, I, I, P]
+        L.oracle_num_threads.restype = I
+        _LIB = L
+    return _LIB
+
+
+def shape_of(wl) -> OrShape:
+    return OrShape(wl.B, wl.Hq, wl.Hkv, wl.Nq, wl.Nkv, wl.d, wl.bq, wl.bk, wl.stride,
+                   1 if wl.paged else 0, wl.num_pages)
+
+
+def _p(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    assert t.device.type == "cpu" and t.is_contiguous()
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _sel(sel: Optional[Sequence]) -> Optional[torch.Tensor]:
+    if sel is None:
+        return None
+    return torch.tensor([list(x) for x in sel], dtype=torch.int32).reshape(-1, 3).contiguous()
+
+
+def num_threads() -> int:
+    return lib().oracle_num_threads()
+
+
+def kmax(wl, budget: float) -> int:
+    return lib().oracle_kmax(ctypes.byref(shape_of(wl)), budget)
+
+
+def causal_blocks(wl, I: int) -> int:
+    return lib().oracle_causal_blocks(ctypes.byref(shape_of(wl)), I)
+
+
+def budget_blocks(n: int, budget: float) -> int:
+    return lib().oracle_budget_blocks(n, budget)
+
+
+def skip_threshold(eps: float, d: int) -> float:
+    return lib().oracle_skip_threshold(eps, d)
+
+
+def pool(x: torch.Tensor, s: int) -> torch.Tensor:
+    """Pool a [rows, d] bf16 matrix with stride s (fp32 token-order sum, x 1/s, bf16 RNE)."""
+    x = x.contiguous()
+    rows, d = x.shape
+    out = torch.empty(rows // s, d, dtype=torch.bfloat16)
+    lib().oracle_pool(_p(x), rows, d, s, _p(out))
+    return out
+
+
+def kap(inp, budget: float, sel=None, kmax_: Optional[int] = None, want_scores: bool = False,
+        threads: int = 0):
+    """Stage 1 (KAP).  Returns dict(order [n,kmax] int32 padded -1, count [n],
+    hrm_count [n], and optionally score [n,nKB] fp32, hrm [n,nKB] uint8).
+    With sel=None, n = B*Hq*nQB in (b, h, I) row-major order."""
+    wl = inp.wl
+    sh = shape_of(wl)
+    km = kmax_ if kmax_ is not None else kmax(wl, budget)
+    selt = _sel(sel)
+    n = selt.shape[0] if selt is not None else wl.B * wl.Hq * wl.n_qblocks
+    order = torch.full((n, max(km, 1)), -1, dtype=torch.int32)
+    count = torch.zeros(n, dtype=torch.int32)
+    hrmc = torch.zeros(n, dtype=torch.int32)
+    score = torch.empty(n, wl.n_kblocks, dtype=torch.float32) if want_scores else None
+    hrm = torch.empty(n, wl.n_kblocks, dtype=torch.uint8) if want_scores else None
+    rc = lib().oracle_kap(ctypes.byref(sh), _p(inp.q.view(torch.int16)), _p(inp.k.view(torch.int16)),
+                          _p(inp.page_table), budget, _p(selt), n if selt is not None else 0,
+                          max(km, 1), _p(order), _p(count), _p(hrmc), _p(score), _p(hrm), threads)
+    if rc != 0:
+        raise ValueError(f"oracle_kap failed ({rc})")
+    out = dict(order=order, count=count, hrm_count=hrmc)
+    if want_scores:
+        out.update(score=score, hrm=hrm)
+    return out
+
+
+def osk(inp, order: torch.Tensor, count: torch.Tensor, eps: float, sel=None, threads: int = 0):
+    """Stage 2 (OSK).  Returns dict(out [n,bq,d] fp64, lse [n,bq] fp64,
+    skipped [n,kmax] uint8)."""
+    wl = inp.wl
+    sh = shape_of(wl)
+    order = order.to(torch.int32).contiguous()
+    count = count.to(torch.int32).contiguous()
+    selt = _sel(sel)
+    n = order.shape[0]
+    km = order.shape[1]
+    out = torch.empty(n, wl.bq, wl.d, dtype=torch.float64)
+    lse = torch.empty(n, wl.bq, dtype=torch.float64)
+    skipped = torch.zeros(n, km, dtype=torch.uint8)
+    rc = lib().oracle_osk(ctypes.byref(sh), _p(inp.q.view(torch.int16)), _p(inp.k.view(torch.int16)),
+                          _p(inp.v.view(torch.int16)), _p(inp.page_table), _p(selt),
+                          n if selt is not None else 0, _p(order), _p(count), km, eps,
+                          _p(out), _p(lse), _p(skipped), threads)
+    if rc != 0:
+        raise ValueError(f"oracle_osk failed ({rc})")
+    return dict(out=out, lse=lse, skipped=skipped)
+
+
+def dense(inp, sel=None, order: Optional[torch.Tensor] = None, count: Optional[torch.Tensor] = None,
+          threads: int = 0):
+    """Textbook causal attention (fp64), optionally restricted to the blocks
+    listed in order/count.  Returns dict(out [n,bq,d], lse [n,bq])."""
+    wl = inp.wl
+    sh = shape_of(wl)
+    selt = _sel(sel)
+    n = selt.shape[0] if selt is not None else wl.B * wl.Hq * wl.n_qblocks
+    km = 0
+    if order is not None:
+        order = order.to(torch.int32).contiguous()
+        count = count.to(torch.int32).contiguous()
+        km = order.shape[1]
+    out = torch.empty(n, wl.bq, wl.d, dtype=torch.float64)
+    lse = torch.empty(n, wl.bq, dtype=torch.float64)
+    rc = lib().oracle_dense(ctypes.byref(sh), _p(inp.q.view(torch.int16)), _p(inp.k.view(torch.int16)),
+                            _p(inp.v.view(torch.int16)), _p(inp.page_table), _p(selt),
+                            n if selt is not None else 0, _p(order), _p(count), km,
+                            _p(out), _p(lse), threads)
+    if rc != 0:
+        raise ValueError(f"oracle_dense failed ({rc})")
+    return dict(out=out, lse=lse)
+
+
+def rows_of(out: torch.Tensor, wl) -> torch.Tensor:
+    """Reshape a full [B*Hq*nQB, bq, d] result into [B, Hq, Nq, d]."""
+    B, Hq, nqb, bq, d = wl.B, wl.Hq, wl.n_qblocks, wl.bq, wl.d
+    return out.view(B, Hq, nqb * bq, d)[:, :, : wl.Nq]
