@@ -1,0 +1,373 @@
+"""Benchmark of the CoSA hot path (KAP plan + OSK attend) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--budget B] [--eps E] [--impl cosa|reference]
+
+One step = one pass of the whole hot path over one batch of synthetic
+input: cosa_plan (kap_pool, kap_score, kap_sort) then cosa_attend
+(osk_attention).  The default workload is the 128K-token GQA layer
+(B=1, 32 query heads, 8 kv heads, d=128, N=131072, blocks of 128, budget
+10%).  Metric: effective TFLOP/s = dense causal attention FLOPs / step time
+(higher is better); ms_per_step is the latency.  Inputs are resident in HBM
+when the timed region starts and exceed L2, so no L2 flush is needed.
+
+N > 1 (torchrun, one rank per GPU): every rank runs its own replica of the
+workload (different seeds) with no data-path collective ("weak" scaling);
+the barrier and max-over-ranks reduction use NCCL.
+
+--impl reference times the CPU oracle (oracle/, plain C + OpenMP, as it
+stands) on a bounded sample of the same workload; rank 0 alone runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "128K-token prefill attention latency & effective TFLOP/s (frac of peak) vs dense"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="gqa_128k", choices=list(synth.WORKLOADS))
+    ap.add_argument("--budget", type=float, default=None)
+    ap.add_argument("--eps", type=float, default=None)
+    ap.add_argument("--impl", default="cosa", choices=["cosa", "reference"])
+    ap.add_argument("--no-dense", action="store_true", help="skip timing the dense path")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), d.get("bf16_tflops_sustained", 1400.0), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.file.flush()
+        rows = []
+        with open(self.file.name) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.file.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------- CPU oracle timing
+
+def oracle_sample(inp, budget, eps, seconds, seed=0):
+    """Run the oracle (KAP + OSK) on (b, h, Q-block) rows drawn from the
+    workload until about `seconds` of wall time.  Returns (dense-equivalent
+    FLOPs of the rows done, seconds, rows, threads)."""
+    import random
+    import oracle
+    wl = inp.wl
+    rng = random.Random(seed)
+    off = wl.Nkv - wl.Nq
+    flops, done, t_all = 0.0, 0, 0.0
+    km = oracle.kmax(wl, budget)
+    while t_all < seconds and done < 4096:
+        sel = [(rng.randrange(wl.B), rng.randrange(wl.Hq), rng.randrange(wl.n_qblocks)) for _ in range(8)]
+        t0 = time.perf_counter()
+        plan = oracle.kap(inp, budget, sel=sel, kmax_=km)
+        oracle.osk(inp, plan["order"], plan["count"], eps, sel=sel)
+        t_all += time.perf_counter() - t0
+        for (_, _, I) in sel:
+            lo, hi = I * wl.bq, min((I + 1) * wl.bq, wl.Nq)
+            pairs = sum(off + i + 1 for i in range(lo, hi))
+            flops += 4.0 * wl.d * pairs
+        done += len(sel)
+    return flops, t_all, done, oracle.num_threads()
+
+
+def run_reference(args, wl, budget, eps):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    inp = synth.generate(wl)
+    per_step = max(2.0, min(12.0, 150.0 / max(1, args.steps + args.warmup)))
+    for w in range(args.warmup):
+        oracle_sample(inp, budget, eps, per_step / 4, seed=100 + w)
+    tot_f, tot_t, rows, thr = 0.0, 0.0, 0, 1
+    for s in range(args.steps):
+        f, t, r, thr = oracle_sample(inp, budget, eps, per_step, seed=s)
+        tot_f, tot_t, rows = tot_f + f, tot_t + t, rows + r
+    value = tot_f / tot_t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "Nq": wl.Nq, "Nkv": wl.Nkv,
+                   "d": wl.d, "bq": wl.bq, "bk": wl.bk, "budget": budget, "eps": eps},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+                         "sample": f"{rows} random (b, head, Q-block) rows of {wl.name}, KAP + OSK each, "
+                                   f"~{per_step:.0f} s per step"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------- GPU arm
+
+def main():
+    args = parse()
+    wl = synth.WORKLOADS[args.workload]
+    budget = args.budget if args.budget is not None else (0.1 if 0.1 in wl.budgets else wl.budgets[0])
+    eps = args.eps if args.eps is not None else wl.eps
+    if args.impl == "reference":
+        run_reference(args, wl, budget, eps)
+        return
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    import block_sparse_attention_kap_b200 as cosa
+
+    # inputs: generated on the host, pinned, copied once to HBM
+    inp = synth.generate(wl, rank=rank)
+    host = [inp.q.pin_memory(), inp.k.pin_memory(), inp.v.pin_memory()]
+    pt_h = inp.page_table.pin_memory() if inp.page_table is not None else None
+    q, k, v = (t.to(dev) for t in host)
+    pt = pt_h.to(dev) if pt_h is not None else None
+    shape = cosa.shape_of_workload(wl)
+    m = cosa.CoSA(shape, device=dev)
+    order, count, hrm = m.alloc_plan(budget)
+    km = order.shape[-1]
+    out = torch.empty(wl.B, wl.Hq, wl.Nq, wl.d, dtype=torch.bfloat16, device=dev)
+    ws = m.workspace()
+    stream = torch.cuda.current_stream()
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def step(timers=None):
+        if timers is not None:
+            timers[0].record(stream)
+        cosa.cosa_plan(shape, q, k, pt, budget, km, order, count, hrm, None, None, ws, m.status, stream)
+        if timers is not None:
+            timers[1].record(stream)
+        cosa.cosa_attend(shape, q, k, v, pt, order, count, km, eps, out, None, None, m.status, stream)
+        if timers is not None:
+            timers[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert m.device_status() == 0, "device status reported a failure"
+
+    # ---------------------------------------------------------- timed region
+    timers = [[ev(), ev(), ev()] for _ in range(args.steps)]
+    t_start, t_end = ev(), ev()
+    with ClockSampler(local) as clk:
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(timers[i])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+    ms_total = t_start.elapsed_time(t_end)
+    kap_ms = statistics.mean(t[0].elapsed_time(t[1]) for t in timers)
+    osk_ms = statistics.mean(t[1].elapsed_time(t[2]) for t in timers)
+    ms_step = ms_total / args.steps
+    if dist is not None:
+        tt = torch.tensor([ms_step, kap_ms, osk_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_step, kap_ms, osk_ms = tt.tolist()
+    clocks = clk.summary()
+
+    # ---------------------------------------------------------- work accounting (outside the timed region)
+    res = m.attend(q, k, v, order, count, eps, page_table=pt, skip_bits=True)
+    torch.cuda.synchronize()
+    sel_blocks = int(count.sum().item())
+    skipped = int(cosa.unpack_skip_bits(res["skip_bits"], km).sum().item())
+    computed = sel_blocks - skipped
+    blk_flops = 2.0 * wl.bq * wl.bk * wl.d
+    osk_flops = blk_flops * (sel_blocks + computed)          # QK for every visited block, PV for computed
+    dense_flops = wl.dense_causal_flops()
+    n_causal = sum(min(wl.n_kblocks, ((wl.Nkv - wl.Nq) + min((I + 1) * wl.bq, wl.Nq) - 1) // wl.bk + 1)
+                   for I in range(wl.n_qblocks)) * wl.B * wl.Hq
+    kap_bytes = 2.0 * wl.d * (wl.B * wl.Hq * wl.Nq + wl.B * wl.Hkv * wl.Nkv) * (1 + 1 / wl.stride) + \
+        4.0 * order.numel() + 8.0 * count.numel()
+
+    hbm_peak, tc_peak, tc_sust, peak_kind = load_peaks()
+    value = world * dense_flops / (ms_step * 1e-3) / 1e12
+    osk_tflops = osk_flops / (osk_ms * 1e-3) / 1e12
+
+    # ---------------------------------------------------------- dense path (same kernel, natural order, eps 0)
+    dense = None
+    if not args.no_dense:
+        d_order, d_count = m.dense_order()
+        dsteps = max(1, min(args.steps, 5))
+        m.attend(q, k, v, d_order, d_count, 0.0, page_table=pt, out=out)
+        torch.cuda.synchronize()
+        a, b = ev(), ev()
+        a.record(stream)
+        for _ in range(dsteps):
+            cosa.cosa_attend(shape, q, k, v, pt, d_order, d_count, d_order.shape[-1], 0.0, out, None, None,
+                             m.status, stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        dense_ms = a.elapsed_time(b) / dsteps
+        if dist is not None:
+            tt = torch.tensor([dense_ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            dense_ms = tt.item()
+        dense = {"ms": dense_ms, "tflops": dense_flops / (dense_ms * 1e-3) / 1e12,
+                 "frac_of_peak": dense_flops / (dense_ms * 1e-3) / 1e12 / tc_peak,
+                 "speedup_of_sparse_step": dense_ms / ms_step}
+        del d_order, d_count
+
+    # ---------------------------------------------------------- end to end through the public API (host buffers)
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host) + (pt_h.numel() * 4 if pt_h is not None else 0)
+    d2h = out.numel() * out.element_size()
+
+    def e2e_step():
+        q.copy_(host[0], non_blocking=True)
+        k.copy_(host[1], non_blocking=True)
+        v.copy_(host[2], non_blocking=True)
+        if pt is not None:
+            pt.copy_(pt_h, non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    esteps = max(1, min(args.steps, 5))
+    a, b = ev(), ev()
+    if dist is not None:
+        dist.barrier()
+    a.record(stream)
+    for _ in range(esteps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(b) / esteps
+    if dist is not None:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = tt.item()
+    assert m.device_status() == 0
+
+    # ---------------------------------------------------------- CPU baseline (rank 0, N = 1)
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        f, t, rows, thr = oracle_sample(inp, budget, eps, args.cpu_seconds)
+        cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+               "sample": f"{rows} random (b, head, Q-block) rows of {wl.name} (KAP + OSK each), {t:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "Nq": wl.Nq, "Nkv": wl.Nkv,
+                       "d": wl.d, "bq": wl.bq, "bk": wl.bk, "stride": wl.stride, "paged": wl.paged,
+                       "budget": budget, "eps": eps, "parallelism": f"replicas x{world}",
+                       "l2": f"inputs larger than L2 ({sum(t.numel() * 2 for t in host) / 1e9:.2f} GB resident), no flush"},
+            "roofline": {"bound": "tensor", "kernel": "osk_attention", "achieved": osk_tflops, "peak": tc_peak,
+                         "unit": "TFLOP/s", "frac": osk_tflops / tc_peak, "traffic": None,
+                         "peak_kind": f"{peak_kind} bf16 dense (burst)",
+                         "algorithmic_flops_per_launch": osk_flops},
+            "kap_roofline": {"bound": "hbm", "kernels": "kap_pool+kap_score+kap_sort", "ms": kap_ms,
+                             "achieved": kap_bytes / (kap_ms * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                             "frac": kap_bytes / (kap_ms * 1e-3) / 1e9 / hbm_peak,
+                             "algorithmic_bytes_per_launch": kap_bytes},
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * dense_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clocks,
+            "kap_ms": kap_ms, "osk_ms": osk_ms,
+            "selected_blocks": sel_blocks, "causal_blocks": n_causal,
+            "selected_frac": sel_blocks / n_causal, "skipped_in_kernel_frac": skipped / max(1, sel_blocks),
+            "dense": dense,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

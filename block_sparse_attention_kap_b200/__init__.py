@@ -1,0 +1,239 @@
+"""Python binding of the CoSA B200 library (libcosa.so, C ABI in include/cosa.h).
+
+Argument marshalling only: torch tensors supply device memory and the
+current CUDA stream; every step of KAP (pooling, scoring, sorting) and OSK
+runs in the library's CUDA kernels.  There is no CPU fallback: importing
+this package without the built library raises ImportError, and every call
+checks the returned cosa_status.
+
+CoSA: "Accelerating Long-Context Inference via Proxy-Kernel Co-Designed
+Sparse Attention" (gist.science/paper/2607.25291), technical summary
+Sec. 2.2 (Kernel-Aware Proxy) and Sec. 2.3 (Ordered-Skipping Kernel).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcosa.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m block_sparse_attention_kap_b200.build` "
+                      "(the CoSA path has no CPU fallback)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+
+class cosa_shape(ctypes.Structure):
+    """Mirror of the C struct cosa_shape."""
+    _fields_ = [(n, ctypes.c_int) for n in
+                ("B", "Hq", "Hkv", "Nq", "Nkv", "d", "bq", "bk", "stride", "paged", "num_pages")]
+
+
+STATUS = {0: "COSA_OK", 1: "COSA_EINVAL", 2: "COSA_EALIGN", 3: "COSA_ESHAPE", 4: "COSA_EWORKSPACE",
+          5: "COSA_ECUDA", 6: "COSA_EUNSUPPORTED"}
+
+
+class CosaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib.cosa_status_string(status).decode()
+        super().__init__(f"{where}: {msg}")
+
+
+_P = ctypes.c_void_p
+_S = ctypes.POINTER(cosa_shape)
+_lib.cosa_num_qblocks.argtypes = [_S]
+_lib.cosa_num_kblocks.argtypes = [_S]
+_lib.cosa_kmax.argtypes = [_S, ctypes.c_double]
+_lib.cosa_plan_workspace_bytes.argtypes = [_S]
+_lib.cosa_plan_workspace_bytes.restype = ctypes.c_size_t
+_lib.cosa_plan.argtypes = [_S, _P, _P, _P, ctypes.c_double, ctypes.c_int, _P, _P, _P, _P, _P, _P,
+                           ctypes.c_size_t, _P, _P]
+_lib.cosa_dense_order.argtypes = [_S, ctypes.c_int, _P, _P, _P]
+_lib.cosa_attend.argtypes = [_S, _P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_double, _P, _P, _P, _P, _P]
+_lib.cosa_skip_threshold.argtypes = [ctypes.c_double, ctypes.c_int]
+_lib.cosa_skip_threshold.restype = ctypes.c_float
+_lib.cosa_status_string.argtypes = [ctypes.c_int]
+_lib.cosa_status_string.restype = ctypes.c_char_p
+
+EXPORTS = ("cosa_num_qblocks", "cosa_num_kblocks", "cosa_kmax", "cosa_plan_workspace_bytes", "cosa_plan",
+           "cosa_dense_order", "cosa_attend", "cosa_skip_threshold", "cosa_status_string", "cosa_version")
+
+
+def make_shape(B, Hq, Hkv, Nq, Nkv, d=128, bq=128, bk=128, stride=16, paged=False, num_pages=0) -> cosa_shape:
+    return cosa_shape(B, Hq, Hkv, Nq, Nkv, d, bq, bk, stride, 1 if paged else 0, num_pages)
+
+
+def _ptr(t: Optional[torch.Tensor], name: str, dtype=None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise CosaError(status, where)
+
+
+# ----------------------------------------------------------------- same names as the C ABI
+
+def cosa_num_qblocks(shape: cosa_shape) -> int:
+    return _lib.cosa_num_qblocks(ctypes.byref(shape))
+
+
+def cosa_num_kblocks(shape: cosa_shape) -> int:
+    return _lib.cosa_num_kblocks(ctypes.byref(shape))
+
+
+def cosa_kmax(shape: cosa_shape, budget: float) -> int:
+    return _lib.cosa_kmax(ctypes.byref(shape), budget)
+
+
+def cosa_plan_workspace_bytes(shape: cosa_shape) -> int:
+    return _lib.cosa_plan_workspace_bytes(ctypes.byref(shape))
+
+
+def cosa_skip_threshold(eps: float, d: int = 128) -> float:
+    return _lib.cosa_skip_threshold(eps, d)
+
+
+def cosa_status_string(status: int) -> str:
+    return _lib.cosa_status_string(status).decode()
+
+
+def cosa_version() -> int:
+    return _lib.cosa_version()
+
+
+def cosa_plan(shape: cosa_shape, q, k, page_table, budget: float, kmax: int, order, count,
+              hrm_count=None, block_score=None, hrm_flags=None, workspace=None, dev_status=None,
+              stream=None) -> None:
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.cosa_plan(ctypes.byref(shape), _ptr(q, "q", torch.bfloat16), _ptr(k, "k", torch.bfloat16),
+                          _ptr(page_table, "page_table", torch.int32), budget, kmax,
+                          _ptr(order, "order", torch.int32), _ptr(count, "count", torch.int32),
+                          _ptr(hrm_count, "hrm_count", torch.int32), _ptr(block_score, "block_score", torch.float32),
+                          _ptr(hrm_flags, "hrm_flags", torch.uint8), _ptr(workspace, "workspace"), ws_bytes,
+                          _ptr(dev_status, "dev_status", torch.int32), _stream(stream)), "cosa_plan")
+
+
+def cosa_dense_order(shape: cosa_shape, kmax: int, order, count, stream=None) -> None:
+    _check(_lib.cosa_dense_order(ctypes.byref(shape), kmax, _ptr(order, "order", torch.int32),
+                                 _ptr(count, "count", torch.int32), _stream(stream)), "cosa_dense_order")
+
+
+def cosa_attend(shape: cosa_shape, q, k, v, page_table, order, count, kmax: int, skip_eps: float, out,
+                lse=None, skip_bits=None, dev_status=None, stream=None) -> None:
+    _check(_lib.cosa_attend(ctypes.byref(shape), _ptr(q, "q", torch.bfloat16), _ptr(k, "k", torch.bfloat16),
+                            _ptr(v, "v", torch.bfloat16), _ptr(page_table, "page_table", torch.int32),
+                            _ptr(order, "order", torch.int32), _ptr(count, "count", torch.int32), kmax, skip_eps,
+                            _ptr(out, "out", torch.bfloat16), _ptr(lse, "lse", torch.float32),
+                            _ptr(skip_bits, "skip_bits", torch.int32), _ptr(dev_status, "dev_status", torch.int32),
+                            _stream(stream)), "cosa_attend")
+
+
+# ----------------------------------------------------------------- convenience (allocation via torch)
+
+class CoSA:
+    """Holds a shape and the KAP workspace; allocates outputs with torch.
+
+    plan(q, k, budget)           -> order [B,Hq,nQB,kmax], count, hrm_count
+    attend(q, k, v, order, count, eps) -> out [B,Hq,Nq,d] (+ lse, skip bits)
+    dense(q, k, v)               -> out of the dense causal path
+    """
+
+    def __init__(self, shape: cosa_shape, device="cuda"):
+        self.shape = shape
+        self.device = torch.device(device)
+        self.nqb = cosa_num_qblocks(shape)
+        self.nkb = cosa_num_kblocks(shape)
+        if self.nqb < 0:
+            raise CosaError(3, "shape")
+        self._ws = None
+        self.status = torch.zeros(1, dtype=torch.int32, device=self.device)
+
+    def workspace(self) -> torch.Tensor:
+        if self._ws is None:
+            nbytes = cosa_plan_workspace_bytes(self.shape)
+            if nbytes == 0:
+                raise CosaError(6, "cosa_plan_workspace_bytes")
+            self._ws = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        return self._ws
+
+    def alloc_plan(self, budget: float):
+        s = self.shape
+        km = max(cosa_kmax(s, budget), 1)
+        order = torch.empty(s.B, s.Hq, self.nqb, km, dtype=torch.int32, device=self.device)
+        count = torch.empty(s.B, s.Hq, self.nqb, dtype=torch.int32, device=self.device)
+        hrm = torch.empty(s.B, s.Hq, self.nqb, dtype=torch.int32, device=self.device)
+        return order, count, hrm
+
+    def plan(self, q, k, budget: float, page_table=None, out=None, scores: bool = False, stream=None):
+        order, count, hrm = out if out is not None else self.alloc_plan(budget)
+        bs = hf = None
+        if scores:
+            s = self.shape
+            bs = torch.empty(s.B, s.Hq, self.nqb, self.nkb, dtype=torch.float32, device=self.device)
+            hf = torch.empty(s.B, s.Hq, self.nqb, self.nkb, dtype=torch.uint8, device=self.device)
+        cosa_plan(self.shape, q, k, page_table, budget, order.shape[-1], order, count, hrm, bs, hf,
+                  self.workspace(), self.status, stream)
+        res = dict(order=order, count=count, hrm_count=hrm)
+        if scores:
+            res.update(block_score=bs, hrm=hf)
+        return res
+
+    def dense_order(self, stream=None):
+        s = self.shape
+        order = torch.empty(s.B, s.Hq, self.nqb, self.nkb, dtype=torch.int32, device=self.device)
+        count = torch.empty(s.B, s.Hq, self.nqb, dtype=torch.int32, device=self.device)
+        cosa_dense_order(s, self.nkb, order, count, stream)
+        return order, count
+
+    def attend(self, q, k, v, order, count, eps: float, page_table=None, out=None, lse: bool = False,
+               skip_bits: bool = False, stream=None):
+        s = self.shape
+        km = order.shape[-1]
+        if out is None:
+            out = torch.empty(s.B, s.Hq, s.Nq, s.d, dtype=torch.bfloat16, device=self.device)
+        lse_t = torch.empty(s.B, s.Hq, s.Nq, dtype=torch.float32, device=self.device) if lse else None
+        sb = torch.empty(s.B, s.Hq, self.nqb, (km + 31) // 32, dtype=torch.int32, device=self.device) \
+            if skip_bits else None
+        cosa_attend(s, q, k, v, page_table, order, count, km, eps, out, lse_t, sb, self.status, stream)
+        return dict(out=out, lse=lse_t, skip_bits=sb)
+
+    def dense(self, q, k, v, page_table=None, stream=None, **kw):
+        order, count = self.dense_order(stream)
+        return self.attend(q, k, v, order, count, 0.0, page_table=page_table, stream=stream, **kw)
+
+    def device_status(self) -> int:
+        return int(self.status.item())
+
+
+def shape_of_workload(wl) -> cosa_shape:
+    return make_shape(wl.B, wl.Hq, wl.Hkv, wl.Nq, wl.Nkv, wl.d, wl.bq, wl.bk, wl.stride, wl.paged,
+                      wl.num_pages if wl.paged else 0)
+
+
+def unpack_skip_bits(bits: torch.Tensor, kmax: int) -> torch.Tensor:
+    """[..., words] int32 -> [..., kmax] uint8 (1 = skipped in-kernel)."""
+    w = bits.to(torch.int64) & 0xFFFFFFFF
+    shifts = torch.arange(32, device=bits.device, dtype=torch.int64)
+    b = (w.unsqueeze(-1) >> shifts) & 1
+    return b.reshape(*bits.shape[:-1], -1)[..., :kmax].to(torch.uint8)

@@ -1,0 +1,79 @@
+// Internal launch interface between the host front end (cosa_api.cu) and
+// the kernels.  Not part of the public C ABI.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace cosa {
+
+constexpr int kD = 128;          // head dimension the kernels implement
+constexpr int kTileRows = 128;   // MMA M (query rows per tile) and pooled rows/keys per KAP tile
+
+// ---------------------------------------------------------------- KAP pooling
+struct PoolParams {
+  const uint16_t* q;            // [B, Hq, Nq, d]
+  const uint16_t* k;            // [B, Hkv, Nkv, d] or paged [P, Hkv, bk, d]
+  const int32_t* page_table;    // [B, nKB] when paged
+  uint16_t* qp;                 // [B, Hq, Nq/s, d]
+  uint16_t* kp;                 // [B, Hkv, Nkv/s, d]
+  int B, Hq, Hkv, Nq, Nkv, s, bk, nkb, paged, num_pages;
+  long long q_items;            // B*Hq*Nq/s pooled rows of Q
+  long long k_items;            // B*Hkv*Nkv/s pooled rows of K
+};
+cudaError_t launch_kap_pool(const PoolParams& p, cudaStream_t st);
+
+// ---------------------------------------------------------------- KAP scoring
+struct ScoreParams {
+  int B, Hq, Hkv, G;
+  int nqp, nkp;                 // pooled rows per head (Nq/s), pooled keys per kv-head (Nkv/s)
+  int off_p;                    // (Nkv - Nq) / s
+  int Nq, Nkv, bq, bk, s;
+  int nqb, nkb;
+  int kpb;                      // pooled keys per KV block (bk / s)
+  int rpq;                      // pooled rows per Q-block (bq / s)
+  int n_row_tiles;              // ceil(nqp / 128)
+  float* rank;                  // [B, Hq, nQB, nKB] ranking key: +1 for HRM blocks, else score
+  float* block_score;           // optional [B, Hq, nQB, nKB]
+  uint8_t* hrm_flags;           // optional [B, Hq, nQB, nKB]
+  uint32_t* status;
+};
+cudaError_t launch_kap_score(const CUtensorMap& tm_qp, const CUtensorMap& tm_kp, const ScoreParams& p,
+                             cudaStream_t st);
+
+// ---------------------------------------------------------------- KAP sort
+struct SortParams {
+  int B, Hq, nqb, nkb, Nq, Nkv, bq, bk;
+  int bp;                       // budget in basis points
+  int kmax;
+  const float* rank;            // [B, Hq, nQB, nKB]
+  int32_t* order;               // [B, Hq, nQB, kmax]
+  int32_t* count;               // [B, Hq, nQB]
+  int32_t* hrm_count;           // optional [B, Hq, nQB]
+  float* block_score;           // optional [B, Hq, nQB, nKB]: -inf written for invisible blocks
+  uint8_t* hrm_flags;           // optional [B, Hq, nQB, nKB]: 0 written for invisible blocks
+};
+cudaError_t launch_kap_sort(const SortParams& p, cudaStream_t st);
+cudaError_t launch_dense_order(int rows, int nqb, int nkb, int Nq, int Nkv, int bq, int bk, int kmax,
+                               int32_t* order, int32_t* count, cudaStream_t st);
+
+// ---------------------------------------------------------------- OSK
+struct OskParams {
+  int B, Hq, Hkv, G, Nq, Nkv, bq, nqb, nkb, paged, num_pages;
+  const int32_t* page_table;    // [B, nKB] when paged
+  const int32_t* order;         // [B, Hq, nQB, kmax]
+  const int32_t* count;         // [B, Hq, nQB]
+  int kmax;
+  float T;                      // skip threshold, raw-logit units (-inf: never skip)
+  float scale_log2;             // log2(e) / sqrt(d)
+  float scale_ln;               // 1 / sqrt(d)
+  uint16_t* out;                // [B, Hq, Nq, d] bf16
+  float* lse;                   // optional [B, Hq, Nq]
+  uint32_t* skip_bits;          // optional [B, Hq, nQB, skip_words]
+  int skip_words;
+  uint32_t* status;
+};
+cudaError_t launch_osk(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                       const OskParams& p, int bk, cudaStream_t st);
+
+}  // namespace cosa

@@ -1,0 +1,223 @@
+// kap_score: the ranking step of the Kernel-Aware Proxy (CoSA technical
+// summary Sec. 2.2, "Block Ranking" and "HRM Flag Generation").
+//
+// One CTA owns 128 pooled query rows of one head.  It streams the pooled
+// keys of the kv-head in tiles of 128 through a TMA ring and contracts them
+// on the tensor cores (tcgen05, bf16 x bf16 -> fp32 in TMEM, two TMEM
+// accumulators so the next tile's MMA overlaps this tile's epilogue):
+//   S[r, c]   = Qp[r] . Kp[c]                    (raw pooled scores)
+//   Bs[r, j]  = max over visible c in block j     (MaxPool over keys)
+// Pass 1 finds each pooled row's max and the first block attaining it
+// (the HRM block).  Pass 2 recomputes the same tiles (bit-identical) and
+// emits, per (Q-block, KV block), the aggregated MaxNorm score
+//   score[I, j] = max over the pooled rows r of I of (Bs[r, j] - rowmax[r])
+// and the HRM flag, packed into one ranking key (+1 for HRM blocks, whose
+// score is 0, else the score <= 0) so the sort needs one array.
+// Recomputing instead of storing Bs keeps the kernel free of a
+// [rows x blocks] scratch buffer; the contraction is cheap next to OSK.
+// Every selection decision (max, subtract, compare) is taken in fp32.
+#include <cuda_bf16.h>
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace cosa {
+
+namespace {
+
+constexpr int kThreads = 160;            // warps 0-3: epilogue (one pooled row each); warp 4: TMA + MMA
+constexpr uint32_t kTileBytes = 128 * 256;   // 128 rows x 128 bf16
+constexpr int kSmemBytes = 3 * kTileBytes + 1024 + 1024;
+
+struct __align__(8) ScoreSmem {
+  uint64_t q_full;
+  uint64_t k_full[2];
+  uint64_t s_full[2];
+  uint64_t s_free[2];
+  uint32_t tmem_base;
+};
+
+// K-major SW128 descriptor of k-step kk (16 bf16) of a 128-row tile stored
+// as two 64-column chunks of 16 KB.
+__device__ __forceinline__ uint64_t tile_desc(uint32_t base, int kk) {
+  return desc_sw128(base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+}
+
+template <int KPB>
+__global__ void __launch_bounds__(kThreads, 2)
+kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constant__ CUtensorMap tm_kp,
+                 const ScoreParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = base;
+  uint8_t* sK = base + kTileBytes;               // two stages
+  ScoreSmem* sm = reinterpret_cast<ScoreSmem*>(base + 3 * kTileBytes);
+
+  // a CTA launched after another one reported a device error does no work
+  const int failed = p.status ? (int)*reinterpret_cast<volatile uint32_t*>(p.status) : 0;
+  if (__syncthreads_or(failed)) return;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int heads = p.Hq * p.B;
+  const int hb = blockIdx.x % heads;
+  const int R = p.n_row_tiles - 1 - blockIdx.x / heads;       // heaviest row tiles first
+  const int h = hb % p.Hq, b = hb / p.Hq, g = h / p.G;
+  const int r_first = R * kTileRows;
+  const int rows_valid = min(kTileRows, p.nqp - r_first);
+  const int cmax = p.off_p + r_first + rows_valid - 1;        // last pooled key any row here can see
+  const int nT = min(cmax / kTileRows + 1, (p.nkp + kTileRows - 1) / kTileRows);
+  const int U = 2 * nT;
+  constexpr int BPT = kTileRows / KPB;                         // KV blocks per key tile
+
+  if (warp == 4) {
+    tmem_alloc(&sm->tmem_base, 256);
+    tmem_relinquish();
+  }
+  if (tid == 128) {
+    mbar_init(&sm->q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm->k_full[i], 1);
+      mbar_init(&sm->s_full[i], 1);
+      mbar_init(&sm->s_free[i], 128);
+    }
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm->tmem_base;
+
+  if (tid == 128) {
+    // ------------------------------------------------ control: TMA + MMA issue
+    tma_prefetch_desc(&tm_qp);
+    tma_prefetch_desc(&tm_kp);
+    const int qp_y = (b * p.Hq + h) * p.nqp + r_first;
+    const int kp_y0 = (b * p.Hkv + g) * p.nkp;
+    mbar_arrive_expect_tx(&sm->q_full, kTileBytes);
+    tma_load_2d(sQ, &tm_qp, &sm->q_full, 0, qp_y);
+    tma_load_2d(sQ + 16384, &tm_qp, &sm->q_full, 64, qp_y);
+    for (int u = 0; u < 2 && u < U; ++u) {
+      uint8_t* dst = sK + u * kTileBytes;
+      const int y = kp_y0 + (u % nT) * kTileRows;
+      mbar_arrive_expect_tx(&sm->k_full[u], kTileBytes);
+      tma_load_2d(dst, &tm_kp, &sm->k_full[u], 0, y);
+      tma_load_2d(dst + 16384, &tm_kp, &sm->k_full[u], 64, y);
+    }
+    bool ok = mbar_wait(&sm->q_full, 0);
+    if (!ok) report(p.status, DEV_TIMEOUT_TMA);
+    const uint32_t idesc = idesc_bf16(128, 128, false, false);
+    const uint32_t q_addr = smem_u32(sQ);
+    for (int u = 0; ok && u < U; ++u) {
+      const int st = u & 1;
+      const uint32_t ph = (u >> 1) & 1;
+      if (!mbar_wait(&sm->k_full[st], ph)) { report(p.status, DEV_TIMEOUT_TMA); break; }
+      if (u >= 2 && !mbar_wait(&sm->s_free[st], ((u >> 1) - 1) & 1)) { report(p.status, DEV_TIMEOUT_PIPE); break; }
+      tc_fence_after();
+      const uint32_t k_addr = smem_u32(sK + st * kTileBytes);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ss(tmem + st * 128, tile_desc(q_addr, kk), tile_desc(k_addr, kk), idesc, kk > 0);
+      tc_commit(&sm->s_full[st]);
+      if (u + 2 < U) {
+        // refill this stage once the MMA that reads it has completed
+        if (!mbar_wait(&sm->s_full[st], ph)) { report(p.status, DEV_TIMEOUT_MMA); break; }
+        uint8_t* dst = sK + st * kTileBytes;
+        const int y = kp_y0 + ((u + 2) % nT) * kTileRows;
+        mbar_arrive_expect_tx(&sm->k_full[st], kTileBytes);
+        tma_load_2d(dst, &tm_kp, &sm->k_full[st], 0, y);
+        tma_load_2d(dst + 16384, &tm_kp, &sm->k_full[st], 64, y);
+      }
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------ epilogue: one pooled row per thread
+    const int r = r_first + tid;
+    const bool row_ok = tid < rows_valid;
+    const int climit = p.off_p + r;
+    const int I = r / p.rpq;
+    const int last_tok = min((I + 1) * p.bq, p.Nq) - 1;
+    const int n_I = min(p.nkb, (p.Nkv - p.Nq + last_tok) / p.bk + 1);
+    const bool qblock_ok = I < p.nqb;
+    const size_t rank_row = ((size_t)(b * p.Hq + h) * p.nqb + I) * p.nkb;
+    const int gl = lane % p.rpq;                // position inside the Q-block's lane group
+    float rowmax = -INFINITY;
+    int argj = -1;
+    for (int u = 0; u < U; ++u) {
+      const int st = u & 1;
+      const int T = u % nT;
+      if (!mbar_wait(&sm->s_full[st], (u >> 1) & 1)) { report(p.status, DEV_TIMEOUT_MMA); break; }
+      tc_fence_after();
+      float bsv[BPT];
+#pragma unroll
+      for (int jj = 0; jj < BPT; ++jj) bsv[jj] = -INFINITY;
+#pragma unroll
+      for (int qc = 0; qc < 4; ++qc) {
+        uint32_t v[32];
+        tmem_ld_x32(tmem_addr(tmem, 32 * warp, st * 128 + 32 * qc), v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int col = 32 * qc + i;
+          const int c = T * kTileRows + col;
+          const bool vis = row_ok && c <= climit && c < p.nkp;
+          const float x = vis ? __uint_as_float(v[i]) : -INFINITY;
+          bsv[col / KPB] = fmaxf(bsv[col / KPB], x);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&sm->s_free[st]);
+      if (u < nT) {
+#pragma unroll
+        for (int jj = 0; jj < BPT; ++jj)
+          if (bsv[jj] > rowmax) { rowmax = bsv[jj]; argj = T * BPT + jj; }
+      } else {
+#pragma unroll
+        for (int jj = 0; jj < BPT; ++jj) {
+          const int j = T * BPT + jj;
+          float z = row_ok ? __fsub_rn(bsv[jj], rowmax) : -INFINITY;
+          if (!row_ok || bsv[jj] == -INFINITY) z = -INFINITY;
+          uint32_t flag = (argj == j) ? 1u : 0u;
+          for (int o = 1; o < p.rpq; o <<= 1) {
+            z = fmaxf(z, __shfl_xor_sync(0xffffffffu, z, o));
+            flag |= __shfl_xor_sync(0xffffffffu, flag, o);
+          }
+          if (qblock_ok && (jj % p.rpq) == gl && j < n_I) {
+            p.rank[rank_row + j] = flag ? 1.0f : z;
+            if (p.block_score) p.block_score[rank_row + j] = z;
+            if (p.hrm_flags) p.hrm_flags[rank_row + j] = (uint8_t)flag;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_kap_score(const CUtensorMap& tm_qp, const CUtensorMap& tm_kp, const ScoreParams& p,
+                             cudaStream_t st) {
+  const unsigned grid = (unsigned)(p.n_row_tiles * p.Hq * p.B);
+  if (grid == 0) return cudaSuccess;
+#define COSA_LAUNCH_SCORE(K)                                                                          \
+  case K: {                                                                                           \
+    cudaError_t e = cudaFuncSetAttribute(kap_score_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                                         kSmemBytes);                                                 \
+    if (e != cudaSuccess) return e;                                                                   \
+    kap_score_kernel<K><<<grid, kThreads, kSmemBytes, st>>>(tm_qp, tm_kp, p);                         \
+    break;                                                                                            \
+  }
+  switch (p.kpb) {
+    COSA_LAUNCH_SCORE(4)
+    COSA_LAUNCH_SCORE(8)
+    COSA_LAUNCH_SCORE(16)
+    COSA_LAUNCH_SCORE(32)
+    default:
+      return cudaErrorInvalidValue;
+  }
+#undef COSA_LAUNCH_SCORE
+  return cudaGetLastError();
+}
+
+}  // namespace cosa

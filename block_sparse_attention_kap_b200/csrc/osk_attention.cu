@@ -1,0 +1,344 @@
+// osk_attention: the Ordered-Skipping Kernel of CoSA (technical summary
+// Sec. 2.3), consuming the computation-order mask M_KAP.
+//
+// One CTA per (batch, query head, Q-block).  It visits only the KV blocks
+// order[0..count-1], in that order ("mask-skipped" blocks are never touched:
+// their tiles are simply never addressed, paged caches are read in place
+// through the page table).  Per visited block:
+//   S = Q K^T          tcgen05 MMA, bf16 x bf16 -> fp32 accumulator in TMEM
+//   m_loc[r]           row max over causally visible keys
+//   skip vote          m_loc = -inf, or m_run finite and m_loc - m_run < T
+//   block skipped      iff all rows vote skip (tile-wide: the "bucket
+//                      effect" of Sec. 1); a skipped block costs QK only
+//   otherwise          online-softmax update (Sec. 2.1), P = exp(...) in
+//                      bf16 written back into TMEM over S, O += P V with P
+//                      read from TMEM and V from shared memory.
+// m_run is the exact running row max over the computed blocks (it drives
+// the skip test); the exponent reference m_scale is refreshed only when the
+// max grows by more than 2^8 in probability terms, so O in TMEM is rarely
+// rescaled.  The result O / l is written as bf16.
+//
+// Roles: warp 4 (one elected thread) issues every TMA load and MMA; warps
+// 0-3 own one query row each (TMEM lane = row).  TMEM: S/P at columns
+// [0, BK), O at [128, 256); 256 columns and < 100 KB of shared memory per
+// CTA, so two CTAs share an SM and one CTA's softmax overlaps the other's
+// tensor-core work.
+#include <cuda_bf16.h>
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace cosa {
+
+namespace {
+
+constexpr int kThreads = 160;
+constexpr uint32_t kQBytes = 128 * 256;
+constexpr uint32_t kDecisionSkip = 1, kDecisionCompute = 2;
+
+template <int BK>
+struct OskCfg {
+  static constexpr uint32_t kKVBytes = BK * 256;           // BK rows x 128 bf16
+  static constexpr uint32_t kChunk = BK * 128;             // one 64-column chunk
+  static constexpr int kSmem = kQBytes + 2 * kKVBytes + 1024 + 1024;
+};
+
+struct __align__(8) OskSmem {
+  uint64_t q_full, k_full, v_full, s_full, p_ready, o_final;
+  uint32_t decision;
+  uint32_t tmem_base;
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Barrier 1 over the 128 softmax threads with an AND reduction.
+__device__ __forceinline__ bool all_rows(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, 1, 128, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&t);
+}
+
+template <int BK>
+__device__ __forceinline__ int kv_row(const OskParams& p, int b, int g, int j) {
+  const int jc = j < 0 ? 0 : (j >= p.nkb ? p.nkb - 1 : j);
+  if (!p.paged) return (b * p.Hkv + g) * p.Nkv + jc * BK;
+  const int page = p.page_table[(size_t)b * p.nkb + jc];
+  return (page * p.Hkv + g) * BK;   // out-of-pool pages land outside the tensor map: zero fill
+}
+
+// 200 registers x 160 threads x 2 CTAs fits the 64K register file.
+template <int BK>
+__global__ void __maxnreg__(200)
+osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const OskParams p) {
+  using Cfg = OskCfg<BK>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = base;
+  uint8_t* sK = base + kQBytes;
+  uint8_t* sV = sK + Cfg::kKVBytes;
+  OskSmem* sm = reinterpret_cast<OskSmem*>(sV + Cfg::kKVBytes);
+
+  const int failed = p.status ? (int)*reinterpret_cast<volatile uint32_t*>(p.status) : 0;
+  if (__syncthreads_or(failed)) return;
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  // heaviest (last) Q-blocks first; the G query heads of a kv-head adjacent
+  int x = blockIdx.x;
+  const int hg = x % p.G; x /= p.G;
+  const int g = x % p.Hkv; x /= p.Hkv;
+  const int b = x % p.B; x /= p.B;
+  const int I = p.nqb - 1 - x;
+  const int h = g * p.G + hg;
+  const size_t row = ((size_t)(b * p.Hq + h)) * p.nqb + I;
+  const int32_t* ord = p.order + row * p.kmax;
+  int n = p.count[row];
+  n = n < 0 ? 0 : (n > p.kmax ? p.kmax : n);
+  const int rows_valid = min(p.bq, p.Nq - I * p.bq);
+
+  if (warp == 4) {
+    tmem_alloc(&sm->tmem_base, 256);
+    tmem_relinquish();
+  }
+  if (tid == 128) {
+    mbar_init(&sm->q_full, 1);
+    mbar_init(&sm->k_full, 1);
+    mbar_init(&sm->v_full, 1);
+    mbar_init(&sm->s_full, 1);
+    mbar_init(&sm->p_ready, 128);
+    mbar_init(&sm->o_final, 1);
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm->tmem_base;
+  const uint32_t tS = tmem, tO = tmem + 128;
+
+  if (tid == 128) {
+    // ------------------------------------------------------------ control thread
+    if (n > 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      const int q_y = (b * p.Hq + h) * p.Nq + I * p.bq;
+      const uint32_t id_qk = idesc_bf16(128, BK, false, false);
+      const uint32_t id_pv = idesc_bf16(128, 128, false, true);
+      const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      auto load_kv = [&](uint8_t* dst, const CUtensorMap* tm, uint64_t* bar, int j) {
+        const int y = kv_row<BK>(p, b, g, j);
+        mbar_arrive_expect_tx(bar, Cfg::kKVBytes);
+        tma_load_2d(dst, tm, bar, 0, y);
+        tma_load_2d(dst + Cfg::kChunk, tm, bar, 64, y);
+      };
+      auto issue_qk = [&]() {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tS, desc_sw128(q_addr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                 desc_sw128(k_addr + (kk >> 2) * Cfg::kChunk + (kk & 3) * 32, 16, 1024), id_qk, kk > 0);
+        tc_commit(&sm->s_full);
+      };
+      mbar_arrive_expect_tx(&sm->q_full, kQBytes);
+      tma_load_2d(sQ, &tm_q, &sm->q_full, 0, q_y);
+      tma_load_2d(sQ + 16384, &tm_q, &sm->q_full, 64, q_y);
+      load_kv(sK, &tm_k, &sm->k_full, ord[0]);
+      load_kv(sV, &tm_v, &sm->v_full, ord[0]);
+      int v_issued = 0;
+      bool any_pv = false, ok = true;
+      if (!mbar_wait(&sm->q_full, 0) || !mbar_wait(&sm->k_full, 0)) { report(p.status, DEV_TIMEOUT_TMA); ok = false; }
+      if (ok) { tc_fence_after(); issue_qk(); }
+      for (int t = 0; ok && t < n; ++t) {
+        const uint32_t ph = t & 1;
+        if (!mbar_wait(&sm->s_full, ph)) { report(p.status, DEV_TIMEOUT_MMA); break; }
+        // QK_t and every earlier MMA are complete: K and V buffers are free
+        if (v_issued < t) { load_kv(sV, &tm_v, &sm->v_full, ord[t]); v_issued = t; }
+        if (t + 1 < n) load_kv(sK, &tm_k, &sm->k_full, ord[t + 1]);
+        if (!mbar_wait(&sm->p_ready, ph)) { report(p.status, DEV_TIMEOUT_PIPE); break; }
+        const uint32_t dec = *reinterpret_cast<volatile uint32_t*>(&sm->decision);
+        if (!mbar_wait(&sm->v_full, ph)) { report(p.status, DEV_TIMEOUT_TMA); break; }
+        if (dec == kDecisionCompute) {
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            mma_ts(tO, tS + kk * 8, desc_sw128(v_addr + kk * 2048, Cfg::kChunk, 1024), id_pv,
+                   (any_pv || kk > 0) ? 1u : 0u);
+          any_pv = true;
+        } else if (t + 1 < n) {
+          load_kv(sV, &tm_v, &sm->v_full, ord[t + 1]);
+          v_issued = t + 1;
+        }
+        if (t + 1 < n) {
+          if (!mbar_wait(&sm->k_full, (t + 1) & 1)) { report(p.status, DEV_TIMEOUT_TMA); break; }
+          tc_fence_after();
+          issue_qk();
+        }
+      }
+      tc_commit(&sm->o_final);
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ softmax rows
+    const int r = tid;
+    const bool row_ok = r < rows_valid;
+    const int qpos = (p.Nkv - p.Nq) + I * p.bq + r;
+    const float sl2 = p.scale_log2;
+    const float tau = 8.0f / sl2;          // refresh the exponent reference past a 2^8 growth
+    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    float m_run = -INFINITY, m_scale = -INFINITY, l = 0.0f;
+    bool any_pv = false;
+    uint32_t skip_word = 0;
+    uint32_t* skip_out = p.skip_bits ? p.skip_bits + row * p.skip_words : nullptr;
+    for (int t = 0; t < n; ++t) {
+      const int j = ord[t];
+      const bool j_ok = j >= 0 && j < p.nkb;
+      if (!mbar_wait(&sm->s_full, t & 1)) { report(p.status, DEV_TIMEOUT_MMA); break; }
+      tc_fence_after();
+      float s[BK];
+#pragma unroll
+      for (int c0 = 0; c0 < BK; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld_x32(tS + lane_base + c0, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[c0 + i] = __uint_as_float(v[i]);
+      }
+      const int lim = min(qpos - j * BK, p.Nkv - 1 - j * BK);   // last visible column
+      if (lim < BK - 1) {
+#pragma unroll
+        for (int c = 0; c < BK; ++c) s[c] = c <= lim ? s[c] : -INFINITY;
+      }
+      float m_loc = s[0];
+#pragma unroll
+      for (int c = 1; c < BK; ++c) m_loc = fmaxf(m_loc, s[c]);
+      const bool vote = !row_ok || !j_ok || m_loc == -INFINITY ||
+                        (m_run != -INFINITY && __fsub_rn(m_loc, m_run) < p.T);
+      const bool skip = all_rows(vote);
+      if (skip) {
+        if (tid == 0) {
+          sm->decision = kDecisionSkip;
+          skip_word |= 1u << (t & 31);
+        }
+      } else {
+        m_run = fmaxf(m_run, m_loc);
+        float alpha = 1.0f;
+        if (m_loc != -INFINITY && (m_scale == -INFINITY || m_loc > m_scale + tau)) {
+          alpha = (m_scale == -INFINITY) ? 0.0f : ex2((m_scale - m_loc) * sl2);
+          m_scale = m_loc;
+        }
+        l *= alpha;
+        // P = exp2((S - m_scale) * log2(e)/sqrt(d)) in bf16 pairs, 64 columns
+        // at a time, over the first BK/2 TMEM columns of S (already read)
+        const float msl = (m_scale == -INFINITY) ? 0.0f : m_scale * sl2;
+        float lsum = 0.0f;
+#pragma unroll
+        for (int c0 = 0; c0 < BK; c0 += 64) {
+          uint32_t w[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float p0 = ex2(fmaf(s[c0 + 2 * i], sl2, -msl));
+            const float p1 = ex2(fmaf(s[c0 + 2 * i + 1], sl2, -msl));
+            // the row sum uses the same bf16-rounded weights the PV product sees
+            const __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
+            const float2 pf = __bfloat1622float2(pr);
+            lsum += pf.x + pf.y;
+            w[i] = *reinterpret_cast<const uint32_t*>(&pr);
+          }
+          tmem_st_x32(tS + lane_base + c0 / 2, w);
+        }
+        l += lsum;
+        if (any_pv && __any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll
+          for (int c0 = 0; c0 < 128; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld_x32(tO + lane_base + c0, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st_x32(tO + lane_base + c0, o);
+          }
+        }
+        if (tid == 0) sm->decision = kDecisionCompute;
+        any_pv = true;
+      }
+      tc_fence_before();
+      mbar_arrive(&sm->p_ready);
+      if (tid == 0 && skip_out && ((t & 31) == 31 || t == n - 1)) {
+        skip_out[t >> 5] = skip_word;
+        skip_word = 0;
+      }
+    }
+    if (tid == 0 && skip_out)
+      for (int w = (n + 31) >> 5; w < p.skip_words; ++w) skip_out[w] = 0;
+    // ------------------------------------------------------------ epilogue
+    bool have_o = any_pv;
+    if (n > 0) {
+      if (!mbar_wait(&sm->o_final, 0)) { report(p.status, DEV_TIMEOUT_MMA); have_o = false; }
+      tc_fence_after();
+    }
+    const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
+    uint16_t* orow = p.out + (((size_t)(b * p.Hq + h)) * p.Nq + (size_t)I * p.bq + r) * kD;
+#pragma unroll
+    for (int c0 = 0; c0 < 128; c0 += 32) {
+      uint32_t o[32];
+      if (have_o) {
+        tmem_ld_x32(tO + lane_base + c0, o);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = 0u;
+      }
+      uint32_t w[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        w[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+      if (row_ok) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+      }
+    }
+    if (row_ok && p.lse)
+      p.lse[((size_t)(b * p.Hq + h)) * p.Nq + (size_t)I * p.bq + r] =
+          l > 0.0f ? m_scale * p.scale_ln + logf(l) : -INFINITY;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+template <int BK>
+cudaError_t launch_bk(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const OskParams& p,
+                      cudaStream_t st) {
+  const unsigned grid = (unsigned)(p.B * p.Hq * p.nqb);
+  if (grid == 0) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(osk_attention_kernel<BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       OskCfg<BK>::kSmem);
+  if (e != cudaSuccess) return e;
+  osk_attention_kernel<BK><<<grid, kThreads, OskCfg<BK>::kSmem, st>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_osk(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                       const OskParams& p, int bk, cudaStream_t st) {
+  if (bk == 128) return launch_bk<128>(tm_q, tm_k, tm_v, p, st);
+  if (bk == 64) return launch_bk<64>(tm_q, tm_k, tm_v, p, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace cosa

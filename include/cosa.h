@@ -1,0 +1,146 @@
+/*
+ * cosa.h -- C ABI of the CoSA block-sparse prefill attention library for
+ * B200 (sm_100a): the Kernel-Aware Proxy (KAP, cosa_plan) and the
+ * Ordered-Skipping Kernel (OSK, cosa_attend).
+ *
+ * Method: "CoSA: Accelerating Long-Context Inference via Proxy-Kernel
+ * Co-Designed Sparse Attention" (gist.science/paper/2607.25291), technical
+ * summary Sec. 2.1 (order invariance, computation-order mask), Sec. 2.2
+ * (KAP), Sec. 2.3 (OSK).  The KV-head-major layout [B, Hkv, L, d] and the
+ * paged-cache form follow "CompactAttention: Accelerating Chunked Prefill
+ * with Block-Union KV Selection" (gist.science/de/paper/2605.16839),
+ * execution stage.
+ *
+ * Conventions for every entry point:
+ *  - All tensor arguments are DEVICE pointers owned by the caller; the
+ *    library allocates no device memory and keeps no pointer after a call
+ *    returns.  Work is enqueued asynchronously on `stream` (0 = legacy
+ *    default stream); outputs are valid once the stream reaches that point.
+ *  - Tensors are dense, row-major, bf16 (uint16 bit patterns) unless stated.
+ *    Q is [B, Hq, Nq, d]; K and V are [B, Hkv, Nkv, d] or, when
+ *    shape->paged, a page pool [num_pages, Hkv, bk, d] addressed through
+ *    page_table [B, ceil(Nkv/bk)] (int32 physical page of each logical KV
+ *    block).  q, k, v and out must be 16-byte aligned.
+ *  - Causality: query i sits at absolute position Nkv - Nq + i and sees keys
+ *    0 .. Nkv - Nq + i.  GQA: query head h reads kv-head h / (Hq / Hkv).
+ *  - Arguments are validated on the host before anything is launched; on
+ *    error nothing is enqueued and a cosa_status other than COSA_OK is
+ *    returned.  Device code never traps: every wait in a kernel is bounded,
+ *    and a timed-out wait writes a nonzero code to *dev_status (optional,
+ *    caller-zeroed uint32 in device memory) before the kernel returns.
+ */
+#ifndef COSA_H
+#define COSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define COSA_API __attribute__((visibility("default")))
+#else
+#define COSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  COSA_OK = 0,
+  COSA_EINVAL = 1,        /* null required pointer or parameter out of range */
+  COSA_EALIGN = 2,        /* a tensor pointer is not 16-byte aligned */
+  COSA_ESHAPE = 3,        /* inconsistent shape (divisibility, Nkv < Nq, ...) */
+  COSA_EWORKSPACE = 4,    /* workspace missing or smaller than cosa_plan_workspace_bytes */
+  COSA_ECUDA = 5,         /* a CUDA runtime/driver call or a launch failed */
+  COSA_EUNSUPPORTED = 6   /* valid but outside what the kernels implement (e.g. d != 128) */
+} cosa_status;
+
+typedef struct {
+  int B, Hq, Hkv;   /* batch, query heads, kv heads (Hq % Hkv == 0) */
+  int Nq, Nkv;      /* query tokens, key tokens (Nkv >= Nq; both multiples of stride) */
+  int d;            /* head dimension; the kernels implement d == 128 */
+  int bq, bk;       /* Q-block rows and KV-block (page) size, each 64 or 128 */
+  int stride;       /* KAP pooling stride s (power of two, s | bq, s | bk, bk/s <= 32, bq/s <= 32) */
+  int paged;        /* 0: K,V are [B,Hkv,Nkv,d]; 1: page pool [num_pages,Hkv,bk,d] + page_table */
+  int num_pages;    /* pages in the pool when paged */
+} cosa_shape;
+
+/* Number of Q-blocks ceil(Nq/bq) and KV blocks ceil(Nkv/bk). */
+COSA_API int cosa_num_qblocks(const cosa_shape* shape);
+COSA_API int cosa_num_kblocks(const cosa_shape* shape);
+
+/* Budget rule (Sec. 2.2 "moderate budget"; the formula is this library's
+ * reading): Q-block I has n_I causally visible KV blocks; KAP keeps
+ * k_I = max(1, ceil(n_I * bp / 10000)) of them, bp = round(budget * 10000).
+ * Returns max over I of k_I: the minimum last dimension of `order` for
+ * cosa_plan.  Returns -1 for an invalid shape or budget outside (0, 1]. */
+COSA_API int cosa_kmax(const cosa_shape* shape, double budget);
+
+/* Bytes of device workspace cosa_plan needs (pooled Q, pooled K and the
+ * per-(head, Q-block) block ranking).  0 for an invalid shape. */
+COSA_API size_t cosa_plan_workspace_bytes(const cosa_shape* shape);
+
+/* KAP, stage 1 (Sec. 2.2): downsample Q and K (mean of `stride` consecutive
+ * tokens), score pooled queries against pooled keys, MaxPool the scores over
+ * the keys of each KV block, MaxNorm each pooled row (subtract its max),
+ * flag HRM blocks (the first block holding a pooled row's max), aggregate
+ * over the pooled rows of each Q-block (max), and sort each Q-block's
+ * causally visible blocks by (HRM desc, score desc, block index asc),
+ * keeping k_I of them.
+ *  order      [B, Hq, nQB, kmax] int32 out: KV block indices in visit
+ *             order, entries >= count padded with -1.
+ *  count      [B, Hq, nQB] int32 out: k_I.
+ *  hrm_count  [B, Hq, nQB] int32 out (nullable): number of HRM blocks.
+ *  block_score [B, Hq, nQB, nKB] fp32 out (nullable): aggregated MaxNorm
+ *             score of every block (-inf where not causally visible).
+ *  hrm_flags  [B, Hq, nQB, nKB] uint8 out (nullable): 1 for HRM blocks.
+ *  workspace  device scratch of ws_bytes >= cosa_plan_workspace_bytes.
+ * Returns COSA_EINVAL if kmax < cosa_kmax(shape, budget). */
+COSA_API cosa_status cosa_plan(const cosa_shape* shape, const void* q, const void* k, const int32_t* page_table,
+                      double budget, int kmax, int32_t* order, int32_t* count, int32_t* hrm_count,
+                      float* block_score, uint8_t* hrm_flags, void* workspace, size_t ws_bytes,
+                      uint32_t* dev_status, cudaStream_t stream);
+
+/* Fill `order`/`count` with every causally visible block of each Q-block in
+ * natural order (0, 1, ..., n_I - 1): the dense path, which cosa_attend runs
+ * with skip_eps = 0 (Sec. 4 reports speedup against dense attention).
+ * kmax must be >= cosa_num_kblocks(shape). */
+COSA_API cosa_status cosa_dense_order(const cosa_shape* shape, int kmax, int32_t* order, int32_t* count,
+                             cudaStream_t stream);
+
+/* OSK, stage 2 (Sec. 2.3): for each (b, h, Q-block I) visit only the KV
+ * blocks order[b,h,I,0..count-1], in that order (mask-skipped blocks are
+ * never touched); per visited block compute S = Q K^T exactly, and skip the
+ * block when every row of the Q-block satisfies m_loc - m_run < T with
+ * T = fp32(ln(skip_eps) * sqrt(d)) in raw-logit units (a row with no visible
+ * key in the block always agrees; the bucket effect of Sec. 1 makes the
+ * decision tile-wide); otherwise update the online softmax (scale
+ * 1/sqrt(d)) and accumulate P V.
+ *  skip_eps   in [0, 1); 0 never skips.
+ *  out        [B, Hq, Nq, d] bf16 out; a row that saw no key is 0.
+ *  lse        [B, Hq, Nq] fp32 out (nullable): log-sum-exp of the scaled
+ *             logits (natural log), -inf for a row that saw no key.
+ *  skip_bits  [B, Hq, nQB, ceil(kmax/32)] uint32 out (nullable): bit t of
+ *             word t/32 set iff visit t was skipped in-kernel.
+ * order entries outside [0, nKB) are treated as skipped blocks; count is
+ * clamped to [0, kmax]. */
+COSA_API cosa_status cosa_attend(const cosa_shape* shape, const void* q, const void* k, const void* v,
+                        const int32_t* page_table, const int32_t* order, const int32_t* count, int kmax,
+                        double skip_eps, void* out, float* lse, uint32_t* skip_bits, uint32_t* dev_status,
+                        cudaStream_t stream);
+
+/* The skip threshold T = fp32(ln(eps) * sqrt(d)) cosa_attend uses (-inf for eps == 0). */
+COSA_API float cosa_skip_threshold(double eps, int d);
+
+/* Human-readable name of a status code (static storage). */
+COSA_API const char* cosa_status_string(cosa_status status);
+
+/* Library ABI version (major * 100 + minor). */
+COSA_API int cosa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* COSA_H */

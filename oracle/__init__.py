@@ -34,7 +34,7 @@ def lib():
         P, I, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
         S = ctypes.POINTER(OrShape)
         L.oracle_kap.argtypes = [S, P, P, P, D, P, I, I, P, P, P, P, P, I]
-        L.oracle_osk.argtypes = [S, P, P, P, P, P, I, P, P, I, D, P, P, P, I]
+        L.oracle_osk.argtypes = [S, P, P, P, P, P, I, P, P, I, D, P, P, P, P, I]
         L.oracle_dense.argtypes = [S, P, P, P, P, P, I, P, P, I, P, P, I]
         L.oracle_kmax.argtypes = [S, D]
         L.oracle_causal_blocks.argtypes = [S, I]
@@ -122,7 +122,8 @@ def kap(inp, budget: float, sel=None, kmax_: Optional[int] = None, want_scores: 
 
 def osk(inp, order: torch.Tensor, count: torch.Tensor, eps: float, sel=None, threads: int = 0):
     """Stage 2 (OSK).  Returns dict(out [n,bq,d] fp64, lse [n,bq] fp64,
-    skipped [n,kmax] uint8)."""
+    skipped [n,kmax] uint8, margin [n,kmax] fp64: per visit the largest row
+    value of fp32(m_loc - m_run) - T, negative iff the block was skipped)."""
     wl = inp.wl
     sh = shape_of(wl)
     order = order.to(torch.int32).contiguous()
@@ -133,13 +134,14 @@ def osk(inp, order: torch.Tensor, count: torch.Tensor, eps: float, sel=None, thr
     out = torch.empty(n, wl.bq, wl.d, dtype=torch.float64)
     lse = torch.empty(n, wl.bq, dtype=torch.float64)
     skipped = torch.zeros(n, km, dtype=torch.uint8)
+    margin = torch.empty(n, km, dtype=torch.float64)
     rc = lib().oracle_osk(ctypes.byref(sh), _p(inp.q.view(torch.int16)), _p(inp.k.view(torch.int16)),
                           _p(inp.v.view(torch.int16)), _p(inp.page_table), _p(selt),
                           n if selt is not None else 0, _p(order), _p(count), km, eps,
-                          _p(out), _p(lse), _p(skipped), threads)
+                          _p(out), _p(lse), _p(skipped), _p(margin), threads)
     if rc != 0:
         raise ValueError(f"oracle_osk failed ({rc})")
-    return dict(out=out, lse=lse, skipped=skipped)
+    return dict(out=out, lse=lse, skipped=skipped, margin=margin)
 
 
 def dense(inp, sel=None, order: Optional[torch.Tensor] = None, count: Optional[torch.Tensor] = None,

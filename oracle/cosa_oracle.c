@@ -332,7 +332,7 @@ float oracle_skip_threshold(double eps, int d) {
 static void osk_one(const or_shape* sh, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                     const int32_t* pt, int b, int h, int I, const int32_t* order, int count,
                     float T, int apply_skip, double* out, double* lse, uint8_t* skipped,
-                    double* qf, double* srow) {
+                    double* margin, double* qf, double* srow) {
     const int d = sh->d, bq = sh->bq, bk = sh->bk, g = h / (sh->Hq / sh->Hkv);
     const int off = sh->Nkv - sh->Nq;
     const int i0 = I * bq;
@@ -349,8 +349,12 @@ static void osk_one(const or_shape* sh, const uint16_t* q, const uint16_t* k, co
     for (int t = 0; t < count; ++t) {
         const int j = order[t];
         const int c0 = j * bk, c1 = (c0 + bk < sh->Nkv ? c0 + bk : sh->Nkv);
-        /* exact logits of the block and the tile-wide skip vote */
+        /* exact logits of the block and the tile-wide skip vote; the block's
+         * margin is the largest row distance above the threshold (< 0 iff
+         * every row votes skip), reported so callers can tell fragile
+         * decisions from robust ones */
         int all_skip = 1;
+        double mg = -INFINITY;
         for (int r = 0; r < nrows; ++r) {
             float m_loc = -INFINITY;
             for (int c = c0; c < c1; ++c) {
@@ -365,9 +369,15 @@ static void osk_one(const or_shape* sh, const uint16_t* q, const uint16_t* k, co
             int vote = (m_loc == -INFINITY) ||
                        (m_run[r] != -INFINITY && (float)(m_loc - m_run[r]) < T);
             if (!vote) all_skip = 0;
+            if (m_loc != -INFINITY) {
+                double dr = (m_run[r] == -INFINITY || T == -INFINITY)
+                                ? INFINITY : (double)(float)(m_loc - m_run[r]) - (double)T;
+                if (dr > mg) mg = dr;
+            }
             srow[(size_t)bk * 256 + r] = m_loc;          /* keep m_loc for the update below */
         }
         if (skipped) skipped[t] = (uint8_t)(apply_skip && all_skip);
+        if (margin) margin[t] = mg;
         if (apply_skip && all_skip) continue;
         for (int r = 0; r < nrows; ++r) {
             float m_loc = (float)srow[(size_t)bk * 256 + r];
@@ -409,12 +419,15 @@ static void osk_one(const or_shape* sh, const uint16_t* q, const uint16_t* k, co
 
 /* Stage 2 over a selection (or everything).  order/count as produced by
  * oracle_kap (or any caller-chosen visit order).  out [n][bq][d], lse
- * [n][bq] (optional), skipped [n][kmax] (optional, 1 = skipped in-kernel).
+ * [n][bq] (optional), skipped [n][kmax] (optional, 1 = skipped in-kernel),
+ * margin [n][kmax] (optional: per visit, the largest row value of
+ * fp32(m_loc - m_run) - T; negative iff the block is skipped, +inf where a
+ * row had no running max yet or eps = 0, -inf where no row saw a key).
  * eps = 0 disables the in-kernel skip. */
 int oracle_osk(const or_shape* sh, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                const int32_t* page_table, const int32_t* sel, int nsel,
                const int32_t* order, const int32_t* count, int kmax, double eps,
-               double* out, double* lse, uint8_t* skipped, int nthreads) {
+               double* out, double* lse, uint8_t* skipped, double* margin, int nthreads) {
     if (check_shape(sh) || sh->bq > 256 || eps < 0.0 || eps >= 1.0) return -1;
     const int n = sel ? nsel : sh->B * sh->Hq * n_qblocks(sh);
     const float T = oracle_skip_threshold(eps, sh->d);
@@ -439,9 +452,11 @@ int oracle_osk(const or_shape* sh, const uint16_t* q, const uint16_t* k, const u
             int b, h, I;
             resolve_sel(sh, sel, nsel, i, &b, &h, &I);
             if (skipped) memset(skipped + (size_t)i * kmax, 0, (size_t)kmax);
+            if (margin) for (int t = 0; t < kmax; ++t) margin[(size_t)i * kmax + t] = NAN;
             osk_one(sh, q, k, v, page_table, b, h, I, order + (size_t)i * kmax, count[i], T, eps > 0.0,
                     out + (size_t)i * sh->bq * sh->d, lse ? lse + (size_t)i * sh->bq : NULL,
-                    skipped ? skipped + (size_t)i * kmax : NULL, qf, srow);
+                    skipped ? skipped + (size_t)i * kmax : NULL, margin ? margin + (size_t)i * kmax : NULL,
+                    qf, srow);
         }
         free(qf);
         free(srow);

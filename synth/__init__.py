@@ -83,7 +83,7 @@ class Workload:
 
     @property
     def num_pages(self) -> int:
-        return self.n_kblocks if self.paged else 0
+        return self.B * self.n_kblocks if self.paged else 0
 
     def dense_causal_flops(self) -> float:
         """4*B*Hq*d*(number of causal (query, key) pairs)."""
