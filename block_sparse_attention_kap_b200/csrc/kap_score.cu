@@ -147,17 +147,23 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
       float bsv[BPT];
 #pragma unroll
       for (int jj = 0; jj < BPT; ++jj) bsv[jj] = -INFINITY;
+      // a tile every column of which this row sees needs no per-column test
+      const bool full = row_ok && T * kTileRows + kTileRows - 1 <= climit && T * kTileRows + kTileRows <= p.nkp;
 #pragma unroll
       for (int qc = 0; qc < 4; ++qc) {
         uint32_t v[32];
         tmem_ld_x32(tmem_addr(tmem, 32 * warp, st * 128 + 32 * qc), v);
+        if (full) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int col = 32 * qc + i;
-          const int c = T * kTileRows + col;
-          const bool vis = row_ok && c <= climit && c < p.nkp;
-          const float x = vis ? __uint_as_float(v[i]) : -INFINITY;
-          bsv[col / KPB] = fmaxf(bsv[col / KPB], x);
+          for (int i = 0; i < 32; ++i) bsv[(32 * qc + i) / KPB] = fmaxf(bsv[(32 * qc + i) / KPB], __uint_as_float(v[i]));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int col = 32 * qc + i;
+            const int c = T * kTileRows + col;
+            const bool vis = row_ok && c <= climit && c < p.nkp;
+            bsv[col / KPB] = fmaxf(bsv[col / KPB], vis ? __uint_as_float(v[i]) : -INFINITY);
+          }
         }
       }
       tc_fence_before();
@@ -167,16 +173,15 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
         for (int jj = 0; jj < BPT; ++jj)
           if (bsv[jj] > rowmax) { rowmax = bsv[jj]; argj = T * BPT + jj; }
       } else {
+        // HRM: the Q-block's flags for this tile, as a bit mask OR-ed over its rows
+        uint32_t bits = (argj >= T * BPT && argj < (T + 1) * BPT) ? 1u << (argj - T * BPT) : 0u;
+        for (int o = 1; o < p.rpq; o <<= 1) bits |= __shfl_xor_sync(0xffffffffu, bits, o);
 #pragma unroll
         for (int jj = 0; jj < BPT; ++jj) {
           const int j = T * BPT + jj;
-          float z = row_ok ? __fsub_rn(bsv[jj], rowmax) : -INFINITY;
-          if (!row_ok || bsv[jj] == -INFINITY) z = -INFINITY;
-          uint32_t flag = (argj == j) ? 1u : 0u;
-          for (int o = 1; o < p.rpq; o <<= 1) {
-            z = fmaxf(z, __shfl_xor_sync(0xffffffffu, z, o));
-            flag |= __shfl_xor_sync(0xffffffffu, flag, o);
-          }
+          float z = (row_ok && bsv[jj] != -INFINITY) ? __fsub_rn(bsv[jj], rowmax) : -INFINITY;
+          for (int o = 1; o < p.rpq; o <<= 1) z = fmaxf(z, __shfl_xor_sync(0xffffffffu, z, o));
+          const uint32_t flag = (bits >> jj) & 1u;
           if (qblock_ok && (jj % p.rpq) == gl && j < n_I) {
             p.rank[rank_row + j] = flag ? 1.0f : z;
             if (p.block_score) p.block_score[rank_row + j] = z;
@@ -204,6 +209,9 @@ cudaError_t launch_kap_score(const CUtensorMap& tm_qp, const CUtensorMap& tm_kp,
   case K: {                                                                                           \
     cudaError_t e = cudaFuncSetAttribute(kap_score_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                                          kSmemBytes);                                                 \
+    if (e != cudaSuccess) return e;                                                                   \
+    e = cudaFuncSetAttribute(kap_score_kernel<K>, cudaFuncAttributePreferredSharedMemoryCarveout,     \
+                             cudaSharedmemCarveoutMaxShared);                                         \
     if (e != cudaSuccess) return e;                                                                   \
     kap_score_kernel<K><<<grid, kThreads, kSmemBytes, st>>>(tm_qp, tm_kp, p);                         \
     break;                                                                                            \

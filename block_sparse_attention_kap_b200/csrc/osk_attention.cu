@@ -35,17 +35,20 @@ constexpr int kThreads = 160;
 constexpr uint32_t kQBytes = 128 * 256;
 constexpr uint32_t kDecisionSkip = 1, kDecisionCompute = 2;
 
+constexpr int kOrderCap = 1024;                            // order entries staged in shared memory
+
 template <int BK>
 struct OskCfg {
   static constexpr uint32_t kKVBytes = BK * 256;           // BK rows x 128 bf16
   static constexpr uint32_t kChunk = BK * 128;             // one 64-column chunk
-  static constexpr int kSmem = kQBytes + 2 * kKVBytes + 1024 + 1024;
+  static constexpr int kSmem = kQBytes + 2 * kKVBytes + 256 + kOrderCap * 4 + 1024;
 };
 
 struct __align__(8) OskSmem {
   uint64_t q_full, k_full, v_full, s_full, p_ready, o_final;
   uint32_t decision;
   uint32_t tmem_base;
+  int32_t order[kOrderCap];     // this CTA's visit order (first kOrderCap entries)
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -81,9 +84,10 @@ __device__ __forceinline__ int kv_row(const OskParams& p, int b, int g, int j) {
   return (page * p.Hkv + g) * BK;   // out-of-pool pages land outside the tensor map: zero fill
 }
 
-// 200 registers x 160 threads x 2 CTAs fits the 64K register file.
+// Two CTAs per SM: 10 warps, so one SM sub-partition holds 3 warps and the
+// kernel must fit in 16K / 3 / 32 = 170 registers per thread.
 template <int BK>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(kThreads, 2)
 osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const OskParams p) {
   using Cfg = OskCfg<BK>;
@@ -111,6 +115,8 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   n = n < 0 ? 0 : (n > p.kmax ? p.kmax : n);
   const int rows_valid = min(p.bq, p.Nq - I * p.bq);
 
+  for (int t = tid; t < n && t < kOrderCap; t += kThreads) sm->order[t] = ord[t];
+  auto order_at = [&](int t) -> int { return t < kOrderCap ? sm->order[t] : ord[t]; };
   if (warp == 4) {
     tmem_alloc(&sm->tmem_base, 256);
     tmem_relinquish();
@@ -156,8 +162,8 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       mbar_arrive_expect_tx(&sm->q_full, kQBytes);
       tma_load_2d(sQ, &tm_q, &sm->q_full, 0, q_y);
       tma_load_2d(sQ + 16384, &tm_q, &sm->q_full, 64, q_y);
-      load_kv(sK, &tm_k, &sm->k_full, ord[0]);
-      load_kv(sV, &tm_v, &sm->v_full, ord[0]);
+      load_kv(sK, &tm_k, &sm->k_full, order_at(0));
+      load_kv(sV, &tm_v, &sm->v_full, order_at(0));
       int v_issued = 0;
       bool any_pv = false, ok = true;
       if (!mbar_wait(&sm->q_full, 0) || !mbar_wait(&sm->k_full, 0)) { report(p.status, DEV_TIMEOUT_TMA); ok = false; }
@@ -166,8 +172,8 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         const uint32_t ph = t & 1;
         if (!mbar_wait(&sm->s_full, ph)) { report(p.status, DEV_TIMEOUT_MMA); break; }
         // QK_t and every earlier MMA are complete: K and V buffers are free
-        if (v_issued < t) { load_kv(sV, &tm_v, &sm->v_full, ord[t]); v_issued = t; }
-        if (t + 1 < n) load_kv(sK, &tm_k, &sm->k_full, ord[t + 1]);
+        if (v_issued < t) { load_kv(sV, &tm_v, &sm->v_full, order_at(t)); v_issued = t; }
+        if (t + 1 < n) load_kv(sK, &tm_k, &sm->k_full, order_at(t + 1));
         if (!mbar_wait(&sm->p_ready, ph)) { report(p.status, DEV_TIMEOUT_PIPE); break; }
         const uint32_t dec = *reinterpret_cast<volatile uint32_t*>(&sm->decision);
         if (!mbar_wait(&sm->v_full, ph)) { report(p.status, DEV_TIMEOUT_TMA); break; }
@@ -179,7 +185,7 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                    (any_pv || kk > 0) ? 1u : 0u);
           any_pv = true;
         } else if (t + 1 < n) {
-          load_kv(sV, &tm_v, &sm->v_full, ord[t + 1]);
+          load_kv(sV, &tm_v, &sm->v_full, order_at(t + 1));
           v_issued = t + 1;
         }
         if (t + 1 < n) {
@@ -203,26 +209,25 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     uint32_t skip_word = 0;
     uint32_t* skip_out = p.skip_bits ? p.skip_bits + row * p.skip_words : nullptr;
     for (int t = 0; t < n; ++t) {
-      const int j = ord[t];
+      const int j = order_at(t);
       const bool j_ok = j >= 0 && j < p.nkb;
       if (!mbar_wait(&sm->s_full, t & 1)) { report(p.status, DEV_TIMEOUT_MMA); break; }
       tc_fence_after();
-      float s[BK];
+      const int lim = min(qpos - j * BK, p.Nkv - 1 - j * BK);   // last visible column
+      // pass 1: row max over the visible columns of S (TMEM -> registers, 32 at a time)
+      float m_loc = -INFINITY;
 #pragma unroll
       for (int c0 = 0; c0 < BK; c0 += 32) {
         uint32_t v[32];
         tmem_ld_x32(tS + lane_base + c0, v);
+        if (lim >= c0 + 31) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[c0 + i] = __uint_as_float(v[i]);
+          for (int i = 0; i < 32; ++i) m_loc = fmaxf(m_loc, __uint_as_float(v[i]));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) m_loc = fmaxf(m_loc, c0 + i <= lim ? __uint_as_float(v[i]) : -INFINITY);
+        }
       }
-      const int lim = min(qpos - j * BK, p.Nkv - 1 - j * BK);   // last visible column
-      if (lim < BK - 1) {
-#pragma unroll
-        for (int c = 0; c < BK; ++c) s[c] = c <= lim ? s[c] : -INFINITY;
-      }
-      float m_loc = s[0];
-#pragma unroll
-      for (int c = 1; c < BK; ++c) m_loc = fmaxf(m_loc, s[c]);
       const bool vote = !row_ok || !j_ok || m_loc == -INFINITY ||
                         (m_run != -INFINITY && __fsub_rn(m_loc, m_run) < p.T);
       const bool skip = all_rows(vote);
@@ -239,17 +244,23 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           m_scale = m_loc;
         }
         l *= alpha;
-        // P = exp2((S - m_scale) * log2(e)/sqrt(d)) in bf16 pairs, 64 columns
-        // at a time, over the first BK/2 TMEM columns of S (already read)
+        // pass 2: P = exp2((S - m_scale) * log2(e)/sqrt(d)), re-read from TMEM 64
+        // columns at a time and written back as bf16 pairs over the first BK/2
+        // columns (all already consumed)
         const float msl = (m_scale == -INFINITY) ? 0.0f : m_scale * sl2;
         float lsum = 0.0f;
 #pragma unroll
         for (int c0 = 0; c0 < BK; c0 += 64) {
+          uint32_t v[64];
+          tmem_ld_x64(tS + lane_base + c0, v);
           uint32_t w[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const float p0 = ex2(fmaf(s[c0 + 2 * i], sl2, -msl));
-            const float p1 = ex2(fmaf(s[c0 + 2 * i + 1], sl2, -msl));
+            const int c = c0 + 2 * i;
+            const float s0 = c <= lim ? __uint_as_float(v[2 * i]) : -INFINITY;
+            const float s1 = c + 1 <= lim ? __uint_as_float(v[2 * i + 1]) : -INFINITY;
+            const float p0 = ex2(fmaf(s0, sl2, -msl));
+            const float p1 = ex2(fmaf(s1, sl2, -msl));
             // the row sum uses the same bf16-rounded weights the PV product sees
             const __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
             const float2 pf = __bfloat1622float2(pr);
@@ -327,6 +338,9 @@ cudaError_t launch_bk(const CUtensorMap& tq, const CUtensorMap& tk, const CUtens
   if (grid == 0) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(osk_attention_kernel<BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        OskCfg<BK>::kSmem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(osk_attention_kernel<BK>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   osk_attention_kernel<BK><<<grid, kThreads, OskCfg<BK>::kSmem, st>>>(tq, tk, tv, p);
   return cudaGetLastError();
