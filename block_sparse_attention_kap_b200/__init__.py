@@ -55,6 +55,7 @@ _lib.cosa_plan_workspace_bytes.restype = ctypes.c_size_t
 _lib.cosa_plan.argtypes = [_S, _P, _P, _P, ctypes.c_double, ctypes.c_int, _P, _P, _P, _P, _P, _P,
                            ctypes.c_size_t, _P, _P]
 _lib.cosa_dense_order.argtypes = [_S, ctypes.c_int, _P, _P, _P]
+_lib.cosa_plan_static.argtypes = [_S, _P, _P, _P, ctypes.c_double, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P]
 _lib.cosa_attend.argtypes = [_S, _P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_double, _P, _P, _P, _P, _P]
 _lib.cosa_skip_threshold.argtypes = [ctypes.c_double, ctypes.c_int]
 _lib.cosa_skip_threshold.restype = ctypes.c_float
@@ -62,7 +63,9 @@ _lib.cosa_status_string.argtypes = [ctypes.c_int]
 _lib.cosa_status_string.restype = ctypes.c_char_p
 
 EXPORTS = ("cosa_num_qblocks", "cosa_num_kblocks", "cosa_kmax", "cosa_plan_workspace_bytes", "cosa_plan",
-           "cosa_dense_order", "cosa_attend", "cosa_skip_threshold", "cosa_status_string", "cosa_version")
+           "cosa_dense_order", "cosa_attend", "cosa_skip_threshold", "cosa_status_string", "cosa_version",
+           "cosa_plan_static")
+STATIC_SCRATCH_BYTES = 64 << 20
 
 
 def make_shape(B, Hq, Hkv, Nq, Nkv, d=128, bq=128, bk=128, stride=16, paged=False, num_pages=0) -> cosa_shape:
@@ -132,6 +135,20 @@ def cosa_plan(shape: cosa_shape, q, k, page_table, budget: float, kmax: int, ord
                           _ptr(hrm_count, "hrm_count", torch.int32), _ptr(block_score, "block_score", torch.float32),
                           _ptr(hrm_flags, "hrm_flags", torch.uint8), _ptr(workspace, "workspace"), ws_bytes,
                           _ptr(dev_status, "dev_status", torch.int32), _stream(stream)), "cosa_plan")
+
+
+def cosa_plan_static(shape: cosa_shape, q, k, page_table, budget: float, kmax: int, order, count,
+                     hrm_count=None, block_score=None, hrm_flags=None, dev_status=None, stream=None) -> None:
+    """cosa_plan for callers that cannot supply a workspace: the scratch is a
+    fixed STATIC_SCRATCH_BYTES array inside the library (shared by all calls;
+    calls that may overlap on the GPU race on it)."""
+    _check(_lib.cosa_plan_static(ctypes.byref(shape), _ptr(q, "q", torch.bfloat16), _ptr(k, "k", torch.bfloat16),
+                                 _ptr(page_table, "page_table", torch.int32), budget, kmax,
+                                 _ptr(order, "order", torch.int32), _ptr(count, "count", torch.int32),
+                                 _ptr(hrm_count, "hrm_count", torch.int32),
+                                 _ptr(block_score, "block_score", torch.float32),
+                                 _ptr(hrm_flags, "hrm_flags", torch.uint8),
+                                 _ptr(dev_status, "dev_status", torch.int32), _stream(stream)), "cosa_plan_static")
 
 
 def cosa_dense_order(shape: cosa_shape, kmax: int, order, count, stream=None) -> None:

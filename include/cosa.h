@@ -130,6 +130,26 @@ COSA_API cosa_status cosa_attend(const cosa_shape* shape, const void* q, const v
                         double skip_eps, void* out, float* lse, uint32_t* skip_bits, uint32_t* dev_status,
                         cudaStream_t stream);
 
+/* cosa_plan without a workspace argument, for callers that cannot obtain
+ * device memory of their own (for example a serving engine that reserves the
+ * whole GPU at start-up and only hands kernels the tensors it owns, or a
+ * plug-in whose host framework keeps the allocator to itself).  The paper has
+ * no counterpart to this call; it exists only for such callers.
+ * Same arguments and results as cosa_plan, minus workspace/ws_bytes.  The
+ * scratch is one fixed array of COSA_STATIC_SCRATCH_BYTES inside the
+ * library's device image: every GPU that loads it holds that memory until the
+ * process exits; shapes with cosa_plan_workspace_bytes(shape) larger than it
+ * get COSA_EWORKSPACE and nothing is launched; calls that can overlap on the
+ * GPU (different streams without ordering) race on the shared array, calls on
+ * one stream do not.  The first call on each device looks up the array's
+ * device address with that device current: make it before any stream
+ * capture.  Nothing is allocated, ever. */
+#define COSA_STATIC_SCRATCH_BYTES (64u << 20)
+COSA_API cosa_status cosa_plan_static(const cosa_shape* shape, const void* q, const void* k,
+                                      const int32_t* page_table, double budget, int kmax, int32_t* order,
+                                      int32_t* count, int32_t* hrm_count, float* block_score,
+                                      uint8_t* hrm_flags, uint32_t* dev_status, cudaStream_t stream);
+
 /* The skip threshold T = fp32(ln(eps) * sqrt(d)) cosa_attend uses (-inf for eps == 0). */
 COSA_API float cosa_skip_threshold(double eps, int d);
 
