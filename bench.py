@@ -52,6 +52,9 @@ def parse():
     ap.add_argument("--no-dense", action="store_true", help="skip timing the dense path")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
+    ap.add_argument("--sweep", action="store_true",
+                    help="one line per budget of the workload: latency, in-kernel skip fraction and error "
+                         "against the dense path (no headline line)")
     return ap.parse_args()
 
 
@@ -174,6 +177,74 @@ def run_reference(args, wl, budget, eps):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------- rank aggregation
+
+def max_over_ranks(values, dist=None, device=None):
+    """Element-wise max of a list of floats over all ranks (the slowest rank
+    sets every time); identity when running on one rank."""
+    if dist is None:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_tflops(flops_per_rank: float, world: int, ms: float) -> float:
+    """Aggregate throughput: the work of all ranks over the slowest rank's time."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
+# ----------------------------------------------------------------- budget sweep
+
+def run_sweep(args, wl, eps):
+    """For every budget of the workload: step latency (plan + attend), the
+    fraction of selected blocks skipped in-kernel, and the error of the
+    sparse output against the dense path on the same inputs."""
+    import block_sparse_attention_kap_b200 as cosa
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    inp = synth.generate(wl)
+    q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
+    pt = inp.page_table.to(dev) if inp.page_table is not None else None
+    shape = cosa.shape_of_workload(wl)
+    m = cosa.CoSA(shape, device=dev)
+    dense_out = m.dense(q, k, v, page_table=pt)["out"].float()
+    stream = torch.cuda.current_stream()
+    dense_flops = wl.dense_causal_flops()
+    for budget in wl.budgets:
+        e = 0.0 if budget >= 1.0 else eps
+        order, count, hrm = m.alloc_plan(budget)
+        km = order.shape[-1]
+        out = torch.empty(wl.B, wl.Hq, wl.Nq, wl.d, dtype=torch.bfloat16, device=dev)
+
+        def step():
+            cosa.cosa_plan(shape, q, k, pt, budget, km, order, count, hrm, None, None, m.workspace(), m.status,
+                           stream)
+            cosa.cosa_attend(shape, q, k, v, pt, order, count, km, e, out, None, None, m.status, stream)
+
+        for _ in range(max(3, args.warmup)):
+            step()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / args.steps
+        res = m.attend(q, k, v, order, count, e, page_table=pt, skip_bits=True)
+        torch.cuda.synchronize()
+        sel = int(count.sum().item())
+        skipped = int(cosa.unpack_skip_bits(res["skip_bits"], km).sum().item())
+        err = (res["out"].float() - dense_out).abs()
+        assert m.device_status() == 0
+        print(json.dumps({
+            "kind": "sweep", "workload": wl.name, "budget": budget, "eps": e, "ms_per_step": ms,
+            "effective_tflops": dense_flops / (ms * 1e-3) / 1e12, "selected_blocks": sel,
+            "skipped_in_kernel_frac": skipped / max(1, sel),
+            "err_vs_dense": {"max_abs": err.max().item(), "mean_abs": err.mean().item()}}), flush=True)
+
+
 # ----------------------------------------------------------------- GPU arm
 
 def main():
@@ -183,6 +254,9 @@ def main():
     eps = args.eps if args.eps is not None else wl.eps
     if args.impl == "reference":
         run_reference(args, wl, budget, eps)
+        return
+    if args.sweep:
+        run_sweep(args, wl, eps)
         return
     if args.warmup < 3:
         args.warmup = 3
@@ -249,10 +323,7 @@ def main():
     kap_ms = statistics.mean(t[0].elapsed_time(t[1]) for t in timers)
     osk_ms = statistics.mean(t[1].elapsed_time(t[2]) for t in timers)
     ms_step = ms_total / args.steps
-    if dist is not None:
-        tt = torch.tensor([ms_step, kap_ms, osk_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_step, kap_ms, osk_ms = tt.tolist()
+    ms_step, kap_ms, osk_ms = max_over_ranks([ms_step, kap_ms, osk_ms], dist, dev)
     clocks = clk.summary()
 
     # ---------------------------------------------------------- work accounting (outside the timed region)
@@ -270,7 +341,7 @@ def main():
         4.0 * order.numel() + 8.0 * count.numel()
 
     hbm_peak, tc_peak, tc_sust, peak_kind = load_peaks()
-    value = world * dense_flops / (ms_step * 1e-3) / 1e12
+    value = whole_job_tflops(dense_flops, world, ms_step)
     osk_tflops = osk_flops / (osk_ms * 1e-3) / 1e12
 
     # ---------------------------------------------------------- dense path (same kernel, natural order, eps 0)
@@ -287,11 +358,7 @@ def main():
                              m.status, stream)
         b.record(stream)
         torch.cuda.synchronize()
-        dense_ms = a.elapsed_time(b) / dsteps
-        if dist is not None:
-            tt = torch.tensor([dense_ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            dense_ms = tt.item()
+        dense_ms = max_over_ranks([a.elapsed_time(b) / dsteps], dist, dev)[0]
         dense = {"ms": dense_ms, "tflops": dense_flops / (dense_ms * 1e-3) / 1e12,
                  "frac_of_peak": dense_flops / (dense_ms * 1e-3) / 1e12 / tc_peak,
                  "speedup_of_sparse_step": dense_ms / ms_step}
@@ -322,11 +389,7 @@ def main():
         e2e_step()
     b.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = a.elapsed_time(b) / esteps
-    if dist is not None:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = tt.item()
+    e2e_ms = max_over_ranks([a.elapsed_time(b) / esteps], dist, dev)[0]
     assert m.device_status() == 0
 
     # ---------------------------------------------------------- CPU baseline (rank 0, N = 1)
@@ -354,7 +417,7 @@ def main():
                              "frac": kap_bytes / (kap_ms * 1e-3) / 1e9 / hbm_peak,
                              "algorithmic_bytes_per_launch": kap_bytes},
             "cpu_baseline": cpu,
-            "e2e": {"value": world * dense_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "e2e": {"value": whole_job_tflops(dense_flops, world, e2e_ms), "unit": "TFLOP/s",
                     "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": 4 * args.steps,
             "clocks": clocks,

@@ -16,6 +16,10 @@
 // Recomputing instead of storing Bs keeps the kernel free of a
 // [rows x blocks] scratch buffer; the contraction is cheap next to OSK.
 // Every selection decision (max, subtract, compare) is taken in fp32.
+//
+// Roles: warp 8 issues TMA and MMA; warps 0-7 are the epilogue, two per TMEM
+// lane quarter (row = 32*(warp%4) + lane), each taking one 64-column half of
+// every tile.  The halves' row maxima are merged once, after pass 1.
 #include <cuda_bf16.h>
 #include "internal.h"
 #include "sm100.cuh"
@@ -24,16 +28,22 @@ namespace cosa {
 
 namespace {
 
-constexpr int kThreads = 160;            // warps 0-3: epilogue (one pooled row each); warp 4: TMA + MMA
-constexpr uint32_t kTileBytes = 128 * 256;   // 128 rows x 128 bf16
-constexpr int kSmemBytes = 3 * kTileBytes + 1024 + 1024;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 32 * (kEpiWarps + 1);
+constexpr int kCtrl = 32 * kEpiWarps;            // the control thread
+constexpr uint32_t kTileBytes = 128 * 256;       // 128 rows x 128 bf16
+constexpr int kSmemBytes = 3 * kTileBytes + 4096 + 1024;
 
 struct __align__(8) ScoreSmem {
   uint64_t q_full;
   uint64_t k_full[2];
   uint64_t s_full[2];
   uint64_t s_free[2];
+  uint64_t drained;
   uint32_t tmem_base;
+  uint32_t abort;
+  float hmax[2][128];                            // pass-1 row maxima of each column half
+  int harg[2][128];                              // ... and the first block attaining them
 };
 
 // K-major SW128 descriptor of k-step kk (16 bf16) of a 128-row tile stored
@@ -51,6 +61,7 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
   uint8_t* sQ = base;
   uint8_t* sK = base + kTileBytes;               // two stages
   ScoreSmem* sm = reinterpret_cast<ScoreSmem*>(base + 3 * kTileBytes);
+  volatile uint32_t* abort = &sm->abort;
 
   // a CTA launched after another one reported a device error does no work
   const int failed = p.status ? (int)*reinterpret_cast<volatile uint32_t*>(p.status) : 0;
@@ -66,18 +77,21 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
   const int nT = min(cmax / kTileRows + 1, (p.nkp + kTileRows - 1) / kTileRows);
   const int U = 2 * nT;
   constexpr int BPT = kTileRows / KPB;                         // KV blocks per key tile
+  constexpr int BPH = BPT / 2;                                 // per 64-column half
 
-  if (warp == 4) {
+  if (warp == kEpiWarps) {
     tmem_alloc(&sm->tmem_base, 256);
     tmem_relinquish();
   }
-  if (tid == 128) {
+  if (tid == kCtrl) {
     mbar_init(&sm->q_full, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm->k_full[i], 1);
       mbar_init(&sm->s_full[i], 1);
-      mbar_init(&sm->s_free[i], 128);
+      mbar_init(&sm->s_free[i], 32 * kEpiWarps);
     }
+    mbar_init(&sm->drained, 1);
+    sm->abort = 0;
     fence_mbar_init();
   }
   tc_fence_before();
@@ -85,7 +99,7 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
   tc_fence_after();
   const uint32_t tmem = sm->tmem_base;
 
-  if (tid == 128) {
+  if (tid == kCtrl) {
     // ------------------------------------------------ control: TMA + MMA issue
     tma_prefetch_desc(&tm_qp);
     tma_prefetch_desc(&tm_kp);
@@ -101,15 +115,14 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
       tma_load_2d(dst, &tm_kp, &sm->k_full[u], 0, y);
       tma_load_2d(dst + 16384, &tm_kp, &sm->k_full[u], 64, y);
     }
-    bool ok = mbar_wait(&sm->q_full, 0);
-    if (!ok) report(p.status, DEV_TIMEOUT_TMA);
+    bool ok = wait_or_abort(&sm->q_full, 0, abort, p.status, DEV_TIMEOUT_TMA);
     const uint32_t idesc = idesc_bf16(128, 128, false, false);
     const uint32_t q_addr = smem_u32(sQ);
     for (int u = 0; ok && u < U; ++u) {
       const int st = u & 1;
       const uint32_t ph = (u >> 1) & 1;
-      if (!mbar_wait(&sm->k_full[st], ph)) { report(p.status, DEV_TIMEOUT_TMA); break; }
-      if (u >= 2 && !mbar_wait(&sm->s_free[st], ((u >> 1) - 1) & 1)) { report(p.status, DEV_TIMEOUT_PIPE); break; }
+      if (!wait_or_abort(&sm->k_full[st], ph, abort, p.status, DEV_TIMEOUT_TMA)) break;
+      if (u >= 2 && !wait_or_abort(&sm->s_free[st], ((u >> 1) - 1) & 1, abort, p.status, DEV_TIMEOUT_PIPE)) break;
       tc_fence_after();
       const uint32_t k_addr = smem_u32(sK + st * kTileBytes);
 #pragma unroll
@@ -118,7 +131,7 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
       tc_commit(&sm->s_full[st]);
       if (u + 2 < U) {
         // refill this stage once the MMA that reads it has completed
-        if (!mbar_wait(&sm->s_full[st], ph)) { report(p.status, DEV_TIMEOUT_MMA); break; }
+        if (!wait_or_abort(&sm->s_full[st], ph, abort, p.status, DEV_TIMEOUT_MMA)) break;
         uint8_t* dst = sK + st * kTileBytes;
         const int y = kp_y0 + ((u + 2) % nT) * kTileRows;
         mbar_arrive_expect_tx(&sm->k_full[st], kTileBytes);
@@ -126,10 +139,15 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
         tma_load_2d(dst + 16384, &tm_kp, &sm->k_full[st], 64, y);
       }
     }
-  } else if (warp < 4) {
-    // ------------------------------------------------ epilogue: one pooled row per thread
-    const int r = r_first + tid;
-    const bool row_ok = tid < rows_valid;
+    // every MMA this thread issued has completed before TMEM is released
+    tc_commit(&sm->drained);
+    mbar_wait(&sm->drained, 0);
+  } else if (warp < kEpiWarps) {
+    // ------------------------------------------------ epilogue: one pooled row, one column half
+    const int quarter = warp & 3, half = warp >> 2;
+    const int row = 32 * quarter + lane;
+    const int r = r_first + row;
+    const bool row_ok = row < rows_valid;
     const int climit = p.off_p + r;
     const int I = r / p.rpq;
     const int last_tok = min((I + 1) * p.bq, p.Nq) - 1;
@@ -142,47 +160,58 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
     for (int u = 0; u < U; ++u) {
       const int st = u & 1;
       const int T = u % nT;
-      if (!mbar_wait(&sm->s_full[st], (u >> 1) & 1)) { report(p.status, DEV_TIMEOUT_MMA); break; }
+      const bool got = wait_or_abort(&sm->s_full[st], (u >> 1) & 1, abort, p.status, DEV_TIMEOUT_MMA);
       tc_fence_after();
-      float bsv[BPT];
+      float bsv[BPH];
 #pragma unroll
-      for (int jj = 0; jj < BPT; ++jj) bsv[jj] = -INFINITY;
-      // a tile every column of which this row sees needs no per-column test
-      const bool full = row_ok && T * kTileRows + kTileRows - 1 <= climit && T * kTileRows + kTileRows <= p.nkp;
+      for (int jh = 0; jh < BPH; ++jh) bsv[jh] = -INFINITY;
+      const int c_lo = T * kTileRows + 64 * half;              // first pooled key of this half
+      // a half every column of which this row sees needs no per-column test
+      const bool full = got && row_ok && c_lo + 63 <= climit && c_lo + 64 <= p.nkp;
 #pragma unroll
-      for (int qc = 0; qc < 4; ++qc) {
+      for (int qc = 0; qc < 2; ++qc) {
         uint32_t v[32];
-        tmem_ld_x32(tmem_addr(tmem, 32 * warp, st * 128 + 32 * qc), v);
+        tmem_ld_x32(tmem_addr(tmem, 32 * quarter, st * 128 + 64 * half + 32 * qc), v);
         if (full) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) bsv[(32 * qc + i) / KPB] = fmaxf(bsv[(32 * qc + i) / KPB], __uint_as_float(v[i]));
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const int col = 32 * qc + i;
-            const int c = T * kTileRows + col;
-            const bool vis = row_ok && c <= climit && c < p.nkp;
-            bsv[col / KPB] = fmaxf(bsv[col / KPB], vis ? __uint_as_float(v[i]) : -INFINITY);
+            const int c = c_lo + 32 * qc + i;
+            const bool vis = got && row_ok && c <= climit && c < p.nkp;
+            bsv[(32 * qc + i) / KPB] = fmaxf(bsv[(32 * qc + i) / KPB], vis ? __uint_as_float(v[i]) : -INFINITY);
           }
         }
       }
       tc_fence_before();
       mbar_arrive(&sm->s_free[st]);
+      const int j0 = T * BPT + half * BPH;                     // first block of this half
       if (u < nT) {
 #pragma unroll
-        for (int jj = 0; jj < BPT; ++jj)
-          if (bsv[jj] > rowmax) { rowmax = bsv[jj]; argj = T * BPT + jj; }
+        for (int jh = 0; jh < BPH; ++jh)
+          if (bsv[jh] > rowmax) { rowmax = bsv[jh]; argj = j0 + jh; }
+        if (u == nT - 1) {
+          // merge the two halves: the larger max; on a tie the smaller block index
+          sm->hmax[half][row] = rowmax;
+          sm->harg[half][row] = argj;
+          named_barrier(1, 32 * kEpiWarps);
+          const float m0 = sm->hmax[0][row], m1 = sm->hmax[1][row];
+          const int a0 = sm->harg[0][row], a1 = sm->harg[1][row];
+          rowmax = fmaxf(m0, m1);
+          argj = (m0 > m1) ? a0 : (m1 > m0) ? a1 : min(a0, a1);
+        }
       } else {
-        // HRM: the Q-block's flags for this tile, as a bit mask OR-ed over its rows
-        uint32_t bits = (argj >= T * BPT && argj < (T + 1) * BPT) ? 1u << (argj - T * BPT) : 0u;
+        // HRM: the Q-block's flags for this half-tile, as a bit mask OR-ed over its rows
+        uint32_t bits = (argj >= j0 && argj < j0 + BPH) ? 1u << (argj - j0) : 0u;
         for (int o = 1; o < p.rpq; o <<= 1) bits |= __shfl_xor_sync(0xffffffffu, bits, o);
 #pragma unroll
-        for (int jj = 0; jj < BPT; ++jj) {
-          const int j = T * BPT + jj;
-          float z = (row_ok && bsv[jj] != -INFINITY) ? __fsub_rn(bsv[jj], rowmax) : -INFINITY;
+        for (int jh = 0; jh < BPH; ++jh) {
+          const int j = j0 + jh;
+          float z = (row_ok && bsv[jh] != -INFINITY) ? __fsub_rn(bsv[jh], rowmax) : -INFINITY;
           for (int o = 1; o < p.rpq; o <<= 1) z = fmaxf(z, __shfl_xor_sync(0xffffffffu, z, o));
-          const uint32_t flag = (bits >> jj) & 1u;
-          if (qblock_ok && (jj % p.rpq) == gl && j < n_I) {
+          const uint32_t flag = (bits >> jh) & 1u;
+          if (qblock_ok && (jh % p.rpq) == gl && j < n_I) {
             p.rank[rank_row + j] = flag ? 1.0f : z;
             if (p.block_score) p.block_score[rank_row + j] = z;
             if (p.hrm_flags) p.hrm_flags[rank_row + j] = (uint8_t)flag;
@@ -193,7 +222,7 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kEpiWarps) {
     tc_fence_after();
     tmem_dealloc(tmem, 256);
   }

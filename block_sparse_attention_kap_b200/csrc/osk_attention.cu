@@ -45,9 +45,10 @@ struct OskCfg {
 };
 
 struct __align__(8) OskSmem {
-  uint64_t q_full, k_full, v_full, s_full, p_ready, o_final;
+  uint64_t q_full, full[2], s_full, decided, p_ready, o_final;
   uint32_t decision;
   uint32_t tmem_base;
+  uint32_t abort;               // set once any wait of this CTA gave up
   int32_t order[kOrderCap];     // this CTA's visit order (first kOrderCap entries)
 };
 
@@ -97,6 +98,7 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   uint8_t* sK = base + kQBytes;
   uint8_t* sV = sK + Cfg::kKVBytes;
   OskSmem* sm = reinterpret_cast<OskSmem*>(sV + Cfg::kKVBytes);
+  volatile uint32_t* abort = &sm->abort;
 
   const int failed = p.status ? (int)*reinterpret_cast<volatile uint32_t*>(p.status) : 0;
   if (__syncthreads_or(failed)) return;
@@ -123,11 +125,13 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   }
   if (tid == 128) {
     mbar_init(&sm->q_full, 1);
-    mbar_init(&sm->k_full, 1);
-    mbar_init(&sm->v_full, 1);
+    mbar_init(&sm->full[0], 1);
+    mbar_init(&sm->full[1], 1);
     mbar_init(&sm->s_full, 1);
+    mbar_init(&sm->decided, 1);
     mbar_init(&sm->p_ready, 128);
     mbar_init(&sm->o_final, 1);
+    sm->abort = 0;
     fence_mbar_init();
   }
   tc_fence_before();
@@ -146,55 +150,75 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       const uint32_t id_qk = idesc_bf16(128, BK, false, false);
       const uint32_t id_pv = idesc_bf16(128, 128, false, true);
       const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-      auto load_kv = [&](uint8_t* dst, const CUtensorMap* tm, uint64_t* bar, int j) {
+      // Two 32 KB buffers ("slots") for K and V tiles.  K of the next visit is
+      // always in flight in the free slot, so a skipped block never waits for
+      // its successor's K; V of a visit is fetched only once the tile-wide vote
+      // says the block is computed, into the slot its K has just vacated,
+      // while the softmax warps are still exponentiating.
+      auto slot = [&](int sl) { return sl ? sV : sK; };
+      auto slot_addr = [&](int sl) { return sl ? v_addr : k_addr; };
+      uint32_t fph = 0u;     // bit sl: parity of the next completion to wait for on slot sl
+      auto load = [&](int sl, const CUtensorMap* tm, int j) {
         const int y = kv_row<BK>(p, b, g, j);
-        mbar_arrive_expect_tx(bar, Cfg::kKVBytes);
-        tma_load_2d(dst, tm, bar, 0, y);
-        tma_load_2d(dst + Cfg::kChunk, tm, bar, 64, y);
+        mbar_arrive_expect_tx(&sm->full[sl], Cfg::kKVBytes);
+        tma_load_2d(slot(sl), tm, &sm->full[sl], 0, y);
+        tma_load_2d(slot(sl) + Cfg::kChunk, tm, &sm->full[sl], 64, y);
       };
-      auto issue_qk = [&]() {
+      auto wait_slot = [&](int sl) {
+        const bool r = wait_or_abort(&sm->full[sl], (fph >> sl) & 1u, abort, p.status, DEV_TIMEOUT_TMA);
+        fph ^= 1u << sl;
+        return r;
+      };
+      auto issue_qk = [&](int sl) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_ss(tS, desc_sw128(q_addr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                 desc_sw128(k_addr + (kk >> 2) * Cfg::kChunk + (kk & 3) * 32, 16, 1024), id_qk, kk > 0);
+                 desc_sw128(slot_addr(sl) + (kk >> 2) * Cfg::kChunk + (kk & 3) * 32, 16, 1024), id_qk, kk > 0);
         tc_commit(&sm->s_full);
       };
       mbar_arrive_expect_tx(&sm->q_full, kQBytes);
       tma_load_2d(sQ, &tm_q, &sm->q_full, 0, q_y);
       tma_load_2d(sQ + 16384, &tm_q, &sm->q_full, 64, q_y);
-      load_kv(sK, &tm_k, &sm->k_full, order_at(0));
-      load_kv(sV, &tm_v, &sm->v_full, order_at(0));
-      int v_issued = 0;
-      bool any_pv = false, ok = true;
-      if (!mbar_wait(&sm->q_full, 0) || !mbar_wait(&sm->k_full, 0)) { report(p.status, DEV_TIMEOUT_TMA); ok = false; }
-      if (ok) { tc_fence_after(); issue_qk(); }
+      load(0, &tm_k, order_at(0));
+      if (n > 1) load(1, &tm_k, order_at(1));
+      bool any_pv = false;
+      bool ok = wait_or_abort(&sm->q_full, 0, abort, p.status, DEV_TIMEOUT_TMA) && wait_slot(0);
+      if (ok) { tc_fence_after(); issue_qk(0); }
+      int ks = 0;            // slot holding K of visit t
+      int pend_k = -1;       // K load deferred until the PV reading its slot has completed
       for (int t = 0; ok && t < n; ++t) {
         const uint32_t ph = t & 1;
-        if (!mbar_wait(&sm->s_full, ph)) { report(p.status, DEV_TIMEOUT_MMA); break; }
-        // QK_t and every earlier MMA are complete: K and V buffers are free
-        if (v_issued < t) { load_kv(sV, &tm_v, &sm->v_full, order_at(t)); v_issued = t; }
-        if (t + 1 < n) load_kv(sK, &tm_k, &sm->k_full, order_at(t + 1));
-        if (!mbar_wait(&sm->p_ready, ph)) { report(p.status, DEV_TIMEOUT_PIPE); break; }
+        const int ns = ks ^ 1;
+        if (!wait_or_abort(&sm->s_full, ph, abort, p.status, DEV_TIMEOUT_MMA)) break;
+        // QK_t and every earlier MMA are complete
+        if (pend_k >= 0) { load(ns, &tm_k, order_at(pend_k)); pend_k = -1; }
+        if (!wait_or_abort(&sm->decided, ph, abort, p.status, DEV_TIMEOUT_PIPE)) break;
         const uint32_t dec = *reinterpret_cast<volatile uint32_t*>(&sm->decision);
-        if (!mbar_wait(&sm->v_full, ph)) { report(p.status, DEV_TIMEOUT_TMA); break; }
         if (dec == kDecisionCompute) {
+          load(ks, &tm_v, order_at(t));
+          if (!wait_or_abort(&sm->p_ready, ph, abort, p.status, DEV_TIMEOUT_PIPE)) break;
+          if (!wait_slot(ks)) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            mma_ts(tO, tS + kk * 8, desc_sw128(v_addr + kk * 2048, Cfg::kChunk, 1024), id_pv,
+            mma_ts(tO, tS + kk * 8, desc_sw128(slot_addr(ks) + kk * 2048, Cfg::kChunk, 1024), id_pv,
                    (any_pv || kk > 0) ? 1u : 0u);
           any_pv = true;
-        } else if (t + 1 < n) {
-          load_kv(sV, &tm_v, &sm->v_full, order_at(t + 1));
-          v_issued = t + 1;
+          if (t + 2 < n) pend_k = t + 2;
+        } else {
+          if (t + 2 < n) load(ks, &tm_k, order_at(t + 2));
+          if (!wait_or_abort(&sm->p_ready, ph, abort, p.status, DEV_TIMEOUT_PIPE)) break;
         }
         if (t + 1 < n) {
-          if (!mbar_wait(&sm->k_full, (t + 1) & 1)) { report(p.status, DEV_TIMEOUT_TMA); break; }
+          if (!wait_slot(ns)) break;
           tc_fence_after();
-          issue_qk();
+          issue_qk(ns);
         }
+        ks = ns;
       }
+      // o_final completes once every MMA issued above has; TMEM is released after it
       tc_commit(&sm->o_final);
+      mbar_wait(&sm->o_final, 0);
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------ softmax rows
@@ -211,32 +235,37 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     for (int t = 0; t < n; ++t) {
       const int j = order_at(t);
       const bool j_ok = j >= 0 && j < p.nkb;
-      if (!mbar_wait(&sm->s_full, t & 1)) { report(p.status, DEV_TIMEOUT_MMA); break; }
+      // after a failure every thread still runs the same barriers, without waiting
+      const bool got = wait_or_abort(&sm->s_full, t & 1, abort, p.status, DEV_TIMEOUT_MMA);
       tc_fence_after();
       const int lim = min(qpos - j * BK, p.Nkv - 1 - j * BK);   // last visible column
-      // pass 1: row max over the visible columns of S (TMEM -> registers, 32 at a time)
-      float m_loc = -INFINITY;
+      // pass 1: row max over the visible columns of S (TMEM -> registers, 32 at a
+      // time), reduced through 4 independent partial maxima
+      float mp[4];
 #pragma unroll
+      for (int i = 0; i < 4; ++i) mp[i] = -INFINITY;
+#pragma unroll 1
       for (int c0 = 0; c0 < BK; c0 += 32) {
         uint32_t v[32];
         tmem_ld_x32(tS + lane_base + c0, v);
         if (lim >= c0 + 31) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) m_loc = fmaxf(m_loc, __uint_as_float(v[i]));
+          for (int i = 0; i < 32; ++i) mp[i & 3] = fmaxf(mp[i & 3], __uint_as_float(v[i]));
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) m_loc = fmaxf(m_loc, c0 + i <= lim ? __uint_as_float(v[i]) : -INFINITY);
+          for (int i = 0; i < 32; ++i) mp[i & 3] = fmaxf(mp[i & 3], c0 + i <= lim ? __uint_as_float(v[i]) : -INFINITY);
         }
       }
-      const bool vote = !row_ok || !j_ok || m_loc == -INFINITY ||
+      const float m_loc = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
+      const bool vote = !got || !row_ok || !j_ok || m_loc == -INFINITY ||
                         (m_run != -INFINITY && __fsub_rn(m_loc, m_run) < p.T);
       const bool skip = all_rows(vote);
-      if (skip) {
-        if (tid == 0) {
-          sm->decision = kDecisionSkip;
-          skip_word |= 1u << (t & 31);
-        }
-      } else {
+      if (tid == 0) {
+        sm->decision = skip ? kDecisionSkip : kDecisionCompute;
+        mbar_arrive(&sm->decided);
+        if (skip) skip_word |= 1u << (t & 31);
+      }
+      if (!skip) {
         m_run = fmaxf(m_run, m_loc);
         float alpha = 1.0f;
         if (m_loc != -INFINITY && (m_scale == -INFINITY || m_loc > m_scale + tau)) {
@@ -244,32 +273,33 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           m_scale = m_loc;
         }
         l *= alpha;
-        // pass 2: P = exp2((S - m_scale) * log2(e)/sqrt(d)), re-read from TMEM 64
+        // pass 2: P = exp2((S - m_scale) * log2(e)/sqrt(d)), re-read from TMEM 32
         // columns at a time and written back as bf16 pairs over the first BK/2
-        // columns (all already consumed)
+        // columns (all already consumed); masked columns only on boundary blocks
         const float msl = (m_scale == -INFINITY) ? 0.0f : m_scale * sl2;
-        float lsum = 0.0f;
+        float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll 1
+        for (int c0 = 0; c0 < BK; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld_x32(tS + lane_base + c0, v);
+          if (lim < c0 + 31) {
 #pragma unroll
-        for (int c0 = 0; c0 < BK; c0 += 64) {
-          uint32_t v[64];
-          tmem_ld_x64(tS + lane_base + c0, v);
-          uint32_t w[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int c = c0 + 2 * i;
-            const float s0 = c <= lim ? __uint_as_float(v[2 * i]) : -INFINITY;
-            const float s1 = c + 1 <= lim ? __uint_as_float(v[2 * i + 1]) : -INFINITY;
-            const float p0 = ex2(fmaf(s0, sl2, -msl));
-            const float p1 = ex2(fmaf(s1, sl2, -msl));
-            // the row sum uses the same bf16-rounded weights the PV product sees
-            const __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
-            const float2 pf = __bfloat1622float2(pr);
-            lsum += pf.x + pf.y;
-            w[i] = *reinterpret_cast<const uint32_t*>(&pr);
+            for (int i = 0; i < 32; ++i)
+              if (c0 + i > lim) v[i] = __float_as_uint(-INFINITY);
           }
-          tmem_st_x32(tS + lane_base + c0 / 2, w);
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float a0 = fmaf(__uint_as_float(v[2 * i]), sl2, -msl);
+            const float a1 = fmaf(__uint_as_float(v[2 * i + 1]), sl2, -msl);
+            const float p0 = ex2(a0);
+            const float p1 = ex2(a1);
+            ls[i & 3] += p0 + p1;
+            w[i] = pack_bf16(p0, p1);
+          }
+          tmem_st_x16(tS + lane_base + c0 / 2, w);
         }
-        l += lsum;
+        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
         if (any_pv && __any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll
           for (int c0 = 0; c0 < 128; c0 += 32) {
@@ -280,7 +310,6 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             tmem_st_x32(tO + lane_base + c0, o);
           }
         }
-        if (tid == 0) sm->decision = kDecisionCompute;
         any_pv = true;
       }
       tc_fence_before();
@@ -295,7 +324,7 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     // ------------------------------------------------------------ epilogue
     bool have_o = any_pv;
     if (n > 0) {
-      if (!mbar_wait(&sm->o_final, 0)) { report(p.status, DEV_TIMEOUT_MMA); have_o = false; }
+      if (!wait_or_abort(&sm->o_final, 0, abort, p.status, DEV_TIMEOUT_MMA)) have_o = false;
       tc_fence_after();
     }
     const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
