@@ -67,6 +67,27 @@ def load_peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch (read + write) of `kernel` on the 128K workload,
+    from the committed ncu record, or None if the record is missing or any
+    source the kernel was built from changed since the capture."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic_gqa_128k.json")
+    try:
+        rec = json.load(open(path))["kernels"][kernel]
+    except (OSError, KeyError, ValueError):
+        return None
+    csrc = os.path.join(ROOT, "block_sparse_attention_kap_b200", "csrc")
+    for fname, digest in rec["sources_sha256_16"].items():
+        try:
+            cur = hashlib.sha256(open(os.path.join(csrc, fname), "rb").read()).hexdigest()[:16]
+        except OSError:
+            return None
+        if cur != digest:
+            return None
+    return rec["dram_read_bytes"] + rec["dram_write_bytes"]
+
+
 # ----------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -409,7 +430,9 @@ def main():
                        "budget": budget, "eps": eps, "parallelism": f"replicas x{world}",
                        "l2": f"inputs larger than L2 ({sum(t.numel() * 2 for t in host) / 1e9:.2f} GB resident), no flush"},
             "roofline": {"bound": "tensor", "kernel": "osk_attention", "achieved": osk_tflops, "peak": tc_peak,
-                         "unit": "TFLOP/s", "frac": osk_tflops / tc_peak, "traffic": None,
+                         "unit": "TFLOP/s", "frac": osk_tflops / tc_peak,
+                         "traffic": recorded_traffic("osk_attention_kernel<128>") if wl.name == "gqa_128k" and
+                         abs(budget - 0.1) < 1e-9 and abs(eps - 1e-4) < 1e-12 and world == 1 else None,
                          "peak_kind": f"{peak_kind} bf16 dense (burst)",
                          "algorithmic_flops_per_launch": osk_flops},
             "kap_roofline": {"bound": "hbm", "kernels": "kap_pool+kap_score+kap_sort", "ms": kap_ms,
