@@ -229,7 +229,8 @@ def run_sweep(args, wl, eps):
     pt = inp.page_table.to(dev) if inp.page_table is not None else None
     shape = cosa.shape_of_workload(wl)
     m = cosa.CoSA(shape, device=dev)
-    dense_out = m.dense(q, k, v, page_table=pt)["out"].float()
+    dense = m.dense(q, k, v, page_table=pt, lse=True)
+    dense_out, dense_lse = dense["out"].float(), dense["lse"]
     stream = torch.cuda.current_stream()
     dense_flops = wl.dense_causal_flops()
     for budget in wl.budgets:
@@ -254,6 +255,10 @@ def run_sweep(args, wl, eps):
         torch.cuda.synchronize()
         ms = a.elapsed_time(b) / args.steps
         res = m.attend(q, k, v, order, count, e, page_table=pt, skip_bits=True)
+        # attention-mass recall of the plan: share of each row's dense softmax
+        # mass inside the selected blocks, exp(lse over them - dense lse)
+        sel_lse = m.attend(q, k, v, order, count, 0.0, page_table=pt, lse=True)["lse"]
+        recall = torch.exp(sel_lse.double() - dense_lse.double())
         torch.cuda.synchronize()
         sel = int(count.sum().item())
         skipped = int(cosa.unpack_skip_bits(res["skip_bits"], km).sum().item())
@@ -263,7 +268,9 @@ def run_sweep(args, wl, eps):
             "kind": "sweep", "workload": wl.name, "budget": budget, "eps": e, "ms_per_step": ms,
             "effective_tflops": dense_flops / (ms * 1e-3) / 1e12, "selected_blocks": sel,
             "skipped_in_kernel_frac": skipped / max(1, sel),
-            "err_vs_dense": {"max_abs": err.max().item(), "mean_abs": err.mean().item()}}), flush=True)
+            "err_vs_dense": {"max_abs": err.max().item(), "mean_abs": err.mean().item()},
+            "mass_recall": {"mean": recall.mean().item(), "p01": torch.quantile(recall.flatten()[::97].float(), 0.01).item(),
+                            "min": recall.min().item()}}), flush=True)
 
 
 # ----------------------------------------------------------------- GPU arm

@@ -32,7 +32,6 @@ constexpr int kEpiWarps = 8;
 constexpr int kThreads = 32 * (kEpiWarps + 1);
 constexpr int kCtrl = 32 * kEpiWarps;            // the control thread
 constexpr uint32_t kTileBytes = 128 * 256;       // 128 rows x 128 bf16
-constexpr int kSmemBytes = 3 * kTileBytes + 4096 + 1024;
 
 struct __align__(8) ScoreSmem {
   uint64_t q_full;
@@ -45,6 +44,10 @@ struct __align__(8) ScoreSmem {
   float hmax[2][128];                            // pass-1 row maxima of each column half
   int harg[2][128];                              // ... and the first block attaining them
 };
+
+// tiles, the control block, and up to 1023 bytes lost aligning the base to 1 KB
+constexpr int kSmemBytes = 3 * kTileBytes + (int)sizeof(ScoreSmem) + 1024;
+static_assert(2 * (kSmemBytes + 1024) <= 228 * 1024, "two CTAs must share an SM");
 
 // K-major SW128 descriptor of k-step kk (16 bf16) of a 128-row tile stored
 // as two 64-column chunks of 16 KB.

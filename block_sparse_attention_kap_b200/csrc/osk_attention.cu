@@ -18,9 +18,13 @@
 // max grows by more than 2^8 in probability terms, so O in TMEM is rarely
 // rescaled.  The result O / l is written as bf16.
 //
-// Roles: warp 4 (one elected thread) issues every TMA load and MMA; warps
-// 0-3 own one query row each (TMEM lane = row).  TMEM: S/P at columns
-// [0, BK), O at [128, 256); 256 columns and < 100 KB of shared memory per
+// Roles: warp 8 (one elected thread) issues every TMA load and MMA; warps
+// 0-7 run the softmax, two threads per query row (TMEM lane = row, warp%4
+// picks the lane quarter, warp/4 the column half).  The skip vote needs no
+// exchange between the halves: fp32 subtraction is monotone, so
+// fp32(m_loc - m_run) < T holds iff it holds for both half maxima; the
+// halves trade maxima only on computed blocks.  TMEM: S/P at columns
+// [0, BK), O at [128, 256); 256 columns and ~104 KB of shared memory per
 // CTA, so two CTAs share an SM and one CTA's softmax overlaps the other's
 // tensor-core work.
 #include <cuda_bf16.h>
@@ -31,18 +35,13 @@ namespace cosa {
 
 namespace {
 
-constexpr int kThreads = 160;
+constexpr int kSoftmaxThreads = 256;                      // 8 warps, two threads per row
+constexpr int kThreads = kSoftmaxThreads + 32;
+constexpr int kCtrl = kSoftmaxThreads;                     // the control thread (warp 8, lane 0)
 constexpr uint32_t kQBytes = 128 * 256;
 constexpr uint32_t kDecisionSkip = 1, kDecisionCompute = 2;
 
 constexpr int kOrderCap = 1024;                            // order entries staged in shared memory
-
-template <int BK>
-struct OskCfg {
-  static constexpr uint32_t kKVBytes = BK * 256;           // BK rows x 128 bf16
-  static constexpr uint32_t kChunk = BK * 128;             // one 64-column chunk
-  static constexpr int kSmem = kQBytes + 2 * kKVBytes + 256 + kOrderCap * 4 + 1024;
-};
 
 struct __align__(8) OskSmem {
   uint64_t q_full, full[2], s_full, decided, p_ready, o_final;
@@ -50,6 +49,17 @@ struct __align__(8) OskSmem {
   uint32_t tmem_base;
   uint32_t abort;               // set once any wait of this CTA gave up
   int32_t order[kOrderCap];     // this CTA's visit order (first kOrderCap entries)
+  float mx[2][128];             // half-row maxima, traded on computed blocks
+  float lx[2][128];             // half-row sums, traded once at the end
+};
+
+template <int BK>
+struct OskCfg {
+  static constexpr uint32_t kKVBytes = BK * 256;           // BK rows x 128 bf16
+  static constexpr uint32_t kChunk = BK * 128;             // one 64-column chunk
+  // tiles, the control block, and up to 1023 bytes lost aligning the base to 1 KB
+  static constexpr int kSmem = kQBytes + 2 * kKVBytes + (int)sizeof(OskSmem) + 1024;
+  static_assert(2 * (kSmem + 1024) <= 228 * 1024, "two CTAs must share an SM");
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -58,13 +68,13 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// Barrier 1 over the 128 softmax threads with an AND reduction.
+// Barrier 1 over the 256 softmax threads with an AND reduction.
 __device__ __forceinline__ bool all_rows(bool v) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred pi, po;\n\t"
       "setp.ne.u32 pi, %1, 0;\n\t"
-      "bar.red.and.pred po, 1, 128, pi;\n\t"
+      "bar.red.and.pred po, 1, 256, pi;\n\t"
       "selp.u32 %0, 1, 0, po;\n\t}"
       : "=r"(r)
       : "r"((uint32_t)v)
@@ -85,8 +95,8 @@ __device__ __forceinline__ int kv_row(const OskParams& p, int b, int g, int j) {
   return (page * p.Hkv + g) * BK;   // out-of-pool pages land outside the tensor map: zero fill
 }
 
-// Two CTAs per SM: 10 warps, so one SM sub-partition holds 3 warps and the
-// kernel must fit in 16K / 3 / 32 = 170 registers per thread.
+// Two CTAs per SM: 18 warps, so one SM sub-partition holds 5 warps and the
+// kernel must fit in 16K / 5 / 32 = 102 registers per thread.
 template <int BK>
 __global__ void __launch_bounds__(kThreads, 2)
 osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -119,17 +129,17 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 
   for (int t = tid; t < n && t < kOrderCap; t += kThreads) sm->order[t] = ord[t];
   auto order_at = [&](int t) -> int { return t < kOrderCap ? sm->order[t] : ord[t]; };
-  if (warp == 4) {
+  if (warp == kCtrl / 32) {
     tmem_alloc(&sm->tmem_base, 256);
     tmem_relinquish();
   }
-  if (tid == 128) {
+  if (tid == kCtrl) {
     mbar_init(&sm->q_full, 1);
     mbar_init(&sm->full[0], 1);
     mbar_init(&sm->full[1], 1);
     mbar_init(&sm->s_full, 1);
     mbar_init(&sm->decided, 1);
-    mbar_init(&sm->p_ready, 128);
+    mbar_init(&sm->p_ready, kSoftmaxThreads);
     mbar_init(&sm->o_final, 1);
     sm->abort = 0;
     fence_mbar_init();
@@ -140,7 +150,7 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   const uint32_t tmem = sm->tmem_base;
   const uint32_t tS = tmem, tO = tmem + 128;
 
-  if (tid == 128) {
+  if (tid == kCtrl) {
     // ------------------------------------------------------------ control thread
     if (n > 0) {
       tma_prefetch_desc(&tm_q);
@@ -201,13 +211,17 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            mma_ts(tO, tS + kk * 8, desc_sw128(slot_addr(ks) + kk * 2048, Cfg::kChunk, 1024), id_pv,
-                   (any_pv || kk > 0) ? 1u : 0u);
+            // P of keys [16kk, 16kk+16): each column half packs its P at the
+            // start of its own S range (TMEM columns half*BK/2 + ...)
+            mma_ts(tO, tS + (kk / (BK / 32)) * (BK / 2) + (kk % (BK / 32)) * 8,
+                   desc_sw128(slot_addr(ks) + kk * 2048, Cfg::kChunk, 1024), id_pv, (any_pv || kk > 0) ? 1u : 0u);
           any_pv = true;
           if (t + 2 < n) pend_k = t + 2;
-        } else {
-          if (t + 2 < n) load(ks, &tm_k, order_at(t + 2));
-          if (!wait_or_abort(&sm->p_ready, ph, abort, p.status, DEV_TIMEOUT_PIPE)) break;
+        } else if (t + 2 < n) {
+          // a skipped block's S was fully read before the vote: the next QK may
+          // overwrite it at once (p_ready of this visit completes before the
+          // next vote, so its phase parity stays in step)
+          load(ks, &tm_k, order_at(t + 2));
         }
         if (t + 1 < n) {
           if (!wait_slot(ns)) break;
@@ -220,15 +234,18 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       tc_commit(&sm->o_final);
       mbar_wait(&sm->o_final, 0);
     }
-  } else if (warp < 4) {
-    // ------------------------------------------------------------ softmax rows
-    const int r = tid;
+  } else if (warp < kSoftmaxThreads / 32) {
+    // ------------------------------------------------------------ softmax: one row, one column half
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = 32 * quarter + (tid & 31);
     const bool row_ok = r < rows_valid;
     const int qpos = (p.Nkv - p.Nq) + I * p.bq + r;
     const float sl2 = p.scale_log2;
     const float tau = 8.0f / sl2;          // refresh the exponent reference past a 2^8 growth
-    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-    float m_run = -INFINITY, m_scale = -INFINITY, l = 0.0f;
+    const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+    constexpr int HC = BK / 2;              // S columns of this half: [c_base, c_base + HC)
+    const int c_base = half * HC;
+    float m_run = -INFINITY, m_scale = -INFINITY, l = 0.0f;   // l: this half's share of the row sum
     bool any_pv = false;
     uint32_t skip_word = 0;
     uint32_t* skip_out = p.skip_bits ? p.skip_bits + row * p.skip_words : nullptr;
@@ -239,13 +256,13 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       const bool got = wait_or_abort(&sm->s_full, t & 1, abort, p.status, DEV_TIMEOUT_MMA);
       tc_fence_after();
       const int lim = min(qpos - j * BK, p.Nkv - 1 - j * BK);   // last visible column
-      // pass 1: row max over the visible columns of S (TMEM -> registers, 32 at a
-      // time), reduced through 4 independent partial maxima
+      // pass 1: max over this half's visible columns (TMEM -> registers, 32 at a
+      // time, 4 independent partial maxima)
       float mp[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) mp[i] = -INFINITY;
 #pragma unroll 1
-      for (int c0 = 0; c0 < BK; c0 += 32) {
+      for (int c0 = c_base; c0 < c_base + HC; c0 += 32) {
         uint32_t v[32];
         tmem_ld_x32(tS + lane_base + c0, v);
         if (lim >= c0 + 31) {
@@ -256,9 +273,10 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           for (int i = 0; i < 32; ++i) mp[i & 3] = fmaxf(mp[i & 3], c0 + i <= lim ? __uint_as_float(v[i]) : -INFINITY);
         }
       }
-      const float m_loc = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
-      const bool vote = !got || !row_ok || !j_ok || m_loc == -INFINITY ||
-                        (m_run != -INFINITY && __fsub_rn(m_loc, m_run) < p.T);
+      const float m_half = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
+      const bool vote = !got || !row_ok || !j_ok || m_half == -INFINITY ||
+                        (m_run != -INFINITY && __fsub_rn(m_half, m_run) < p.T);
+      tc_fence_before();                  // S reads are ordered before the hand-off below
       const bool skip = all_rows(vote);
       if (tid == 0) {
         sm->decision = skip ? kDecisionSkip : kDecisionCompute;
@@ -266,6 +284,9 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         if (skip) skip_word |= 1u << (t & 31);
       }
       if (!skip) {
+        sm->mx[half][r] = m_half;
+        named_barrier(2, kSoftmaxThreads);
+        const float m_loc = fmaxf(sm->mx[0][r], sm->mx[1][r]);
         m_run = fmaxf(m_run, m_loc);
         float alpha = 1.0f;
         if (m_loc != -INFINITY && (m_scale == -INFINITY || m_loc > m_scale + tau)) {
@@ -273,41 +294,41 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           m_scale = m_loc;
         }
         l *= alpha;
-        // pass 2: P = exp2((S - m_scale) * log2(e)/sqrt(d)), re-read from TMEM 32
-        // columns at a time and written back as bf16 pairs over the first BK/2
-        // columns (all already consumed); masked columns only on boundary blocks
+        // pass 2: P = exp2((S - m_scale) * log2(e)/sqrt(d)) over this half's
+        // columns, re-read 16 at a time and written back as bf16 pairs into
+        // TMEM columns [c_base, c_base + HC/2): inside this half's own S range
+        // and behind its reads, so the other half's S is never overwritten
         const float msl = (m_scale == -INFINITY) ? 0.0f : m_scale * sl2;
         float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll 1
-        for (int c0 = 0; c0 < BK; c0 += 32) {
-          uint32_t v[32];
-          tmem_ld_x32(tS + lane_base + c0, v);
-          if (lim < c0 + 31) {
+        for (int c0 = c_base; c0 < c_base + HC; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld_x16(tS + lane_base + c0, v);
+          if (lim < c0 + 15) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
+            for (int i = 0; i < 16; ++i)
               if (c0 + i > lim) v[i] = __float_as_uint(-INFINITY);
           }
-          uint32_t w[16];
+          uint32_t w[8];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float a0 = fmaf(__uint_as_float(v[2 * i]), sl2, -msl);
-            const float a1 = fmaf(__uint_as_float(v[2 * i + 1]), sl2, -msl);
-            const float p0 = ex2(a0);
-            const float p1 = ex2(a1);
+          for (int i = 0; i < 8; ++i) {
+            const float p0 = ex2(fmaf(__uint_as_float(v[2 * i]), sl2, -msl));
+            const float p1 = ex2(fmaf(__uint_as_float(v[2 * i + 1]), sl2, -msl));
             ls[i & 3] += p0 + p1;
             w[i] = pack_bf16(p0, p1);
           }
-          tmem_st_x16(tS + lane_base + c0 / 2, w);
+          tmem_st_x8(tS + lane_base + c_base + (c0 - c_base) / 2, w);
         }
         l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        // rescale this half of O when the exponent reference moved
         if (any_pv && __any_sync(0xffffffffu, alpha != 1.0f)) {
-#pragma unroll
-          for (int c0 = 0; c0 < 128; c0 += 32) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < 64; c0 += 32) {
             uint32_t o[32];
-            tmem_ld_x32(tO + lane_base + c0, o);
+            tmem_ld_x32(tO + lane_base + 64 * half + c0, o);
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st_x32(tO + lane_base + c0, o);
+            tmem_st_x32(tO + lane_base + 64 * half + c0, o);
           }
         }
         any_pv = true;
@@ -327,13 +348,16 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       if (!wait_or_abort(&sm->o_final, 0, abort, p.status, DEV_TIMEOUT_MMA)) have_o = false;
       tc_fence_after();
     }
-    const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
-    uint16_t* orow = p.out + (((size_t)(b * p.Hq + h)) * p.Nq + (size_t)I * p.bq + r) * kD;
-#pragma unroll
-    for (int c0 = 0; c0 < 128; c0 += 32) {
+    sm->lx[half][r] = l;
+    named_barrier(2, kSoftmaxThreads);
+    const float l_row = sm->lx[0][r] + sm->lx[1][r];
+    const float inv_l = l_row > 0.0f ? 1.0f / l_row : 0.0f;
+    uint16_t* orow = p.out + (((size_t)(b * p.Hq + h)) * p.Nq + (size_t)I * p.bq + r) * kD + 64 * half;
+#pragma unroll 1
+    for (int c0 = 0; c0 < 64; c0 += 32) {
       uint32_t o[32];
       if (have_o) {
-        tmem_ld_x32(tO + lane_base + c0, o);
+        tmem_ld_x32(tO + lane_base + 64 * half + c0, o);
       } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] = 0u;
@@ -348,13 +372,13 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
       }
     }
-    if (row_ok && p.lse)
+    if (row_ok && half == 0 && p.lse)
       p.lse[((size_t)(b * p.Hq + h)) * p.Nq + (size_t)I * p.bq + r] =
-          l > 0.0f ? m_scale * p.scale_ln + logf(l) : -INFINITY;
+          l_row > 0.0f ? m_scale * p.scale_ln + logf(l_row) : -INFINITY;
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kCtrl / 32) {
     tc_fence_after();
     tmem_dealloc(tmem, 256);
   }

@@ -315,3 +315,23 @@ def test_full_size_sampled(cosa, name, budget):
     res = gpu_attend(m, dev, order.view_as(plan["order"]), count.view_as(plan["count"]), EPS)
     o = oracle.osk(inp, ref["order"], ref["count"], EPS, sel=sel)
     check_skips_and_out(cosa, res, o, wl, km, sel_idx=idx)
+
+
+def test_mass_recall_matches_oracle(cosa):
+    """Attention-mass recall of M_KAP (fraction of each row's dense softmax
+    mass inside the selected blocks) from the GPU's log-sum-exp outputs:
+    exp(lse of OSK on the KAP order with eps 0 - lse of the dense path)."""
+    wl = synth.WORKLOADS["gqa_32k"].replace(Nq=4096, Nkv=4096, Hq=4, Hkv=1, n_needle=4)
+    inp = synth.generate(wl)
+    ref_plan = oracle.kap(inp, 0.2)
+    m, dev, _ = gpu_plan(cosa, inp, 0.2, scores=False)
+    order = ref_plan["order"].view(wl.B, wl.Hq, wl.n_qblocks, -1).cuda()
+    count = ref_plan["count"].view(wl.B, wl.Hq, wl.n_qblocks).cuda()
+    sel = gpu_attend(m, dev, order, count, 0.0)
+    dense = m.dense(*dev[:3], lse=True)
+    torch.cuda.synchronize()
+    rec_gpu = torch.exp(sel["lse"].double() - dense["lse"].double()).cpu().view(-1, wl.bq)
+    rec_ref = torch.exp(oracle.dense(inp, order=ref_plan["order"], count=ref_plan["count"])["lse"] -
+                        oracle.dense(inp)["lse"])
+    # each lse is within LSE_TOL of the exact value, so the ratio within ~2*LSE_TOL relative
+    assert torch.allclose(rec_gpu, rec_ref, rtol=2 * LSE_TOL, atol=0)

@@ -413,3 +413,37 @@ def test_skip_decisions_bruteforce_grid():
                 assert res["skipped"][i, t].item() == int(skip)
                 if not skip:
                     m_run = np.maximum(m_run, m_loc)
+
+
+# ----------------------------------------------------------------- attention-mass recall of M_KAP
+
+def test_mass_recall_identity():
+    """The fraction of a row's dense softmax mass inside the selected blocks
+    (the block attention mass m_b = sum over the block's keys of
+    exp(q.k / sqrt(d)), normalised by the row total) equals
+    exp(lse_selected - lse_dense).  Block masses come from a direct fp64
+    matmul here; the lse values from the oracle's dense routine."""
+    wl = tiny(Hq=2, Hkv=1, Nq=256, Nkv=384, bq=64, bk=64, structured=True, n_needle=1)
+    inp = synth.generate(wl)
+    plan = oracle.kap(inp, 0.3)
+    dense = oracle.dense(inp)
+    sel = oracle.dense(inp, order=plan["order"], count=plan["count"])
+    recall = torch.exp(sel["lse"] - dense["lse"])                      # [n, bq]
+    q = inp.q.double()
+    k = inp.k.double()
+    off = wl.Nkv - wl.Nq
+    i = 0
+    for h in range(wl.Hq):
+        s = (q[0, h] @ k[0, 0].T) / math.sqrt(wl.d)                     # [Nq, Nkv]
+        pos = torch.arange(wl.Nq)[:, None] + off
+        s[torch.arange(wl.Nkv)[None, :] > pos] = -math.inf
+        w = torch.softmax(s, dim=-1)
+        for I in range(wl.n_qblocks):
+            chosen = plan["order"][i, : plan["count"][i]].tolist()
+            cols = torch.zeros(wl.Nkv, dtype=torch.bool)
+            for j in chosen:
+                cols[j * wl.bk:(j + 1) * wl.bk] = True
+            mass = w[I * wl.bq:(I + 1) * wl.bq][:, cols].sum(-1)
+            assert torch.allclose(recall[i], mass, atol=1e-12, rtol=1e-9)
+            i += 1
+    assert bool((recall <= 1 + 1e-12).all()) and bool((recall > 0).all())
