@@ -94,7 +94,7 @@ int budget_k(int n, int bp) {
 }
 
 struct Workspace {
-  size_t qp, kp, rank, total;
+  size_t qp, kp, rank, bs, total;
 };
 
 Workspace carve(const cosa_shape* s) {
@@ -104,7 +104,9 @@ Workspace carve(const cosa_shape* s) {
   w.qp = 0;
   w.kp = align256(w.qp + (size_t)rows_q * kD * 2);
   w.rank = align256(w.kp + (size_t)rows_k * kD * 2);
-  w.total = align256(w.rank + (size_t)s->B * s->Hq * n_qblocks(s) * n_kblocks(s) * sizeof(float));
+  w.bs = align256(w.rank + (size_t)s->B * s->Hq * n_qblocks(s) * n_kblocks(s) * sizeof(float));
+  const size_t row_tiles = (size_t)cdiv(s->Nq / s->stride, kTileRows);
+  w.total = align256(w.bs + (size_t)s->B * s->Hq * row_tiles * n_kblocks(s) * kTileRows * sizeof(float));
   return w;
 }
 
@@ -153,6 +155,7 @@ cosa_status cosa_plan(const cosa_shape* shape, const void* q, const void* k, con
   uint16_t* qp = reinterpret_cast<uint16_t*>(ws + w.qp);
   uint16_t* kp = reinterpret_cast<uint16_t*>(ws + w.kp);
   float* rank = reinterpret_cast<float*>(ws + w.rank);
+  float* bs = reinterpret_cast<float*>(ws + w.bs);
   const int str = s.stride;
 
   PoolParams pp;
@@ -177,7 +180,7 @@ cosa_status cosa_plan(const cosa_shape* shape, const void* q, const void* k, con
   sp.nqb = n_qblocks(&s); sp.nkb = n_kblocks(&s);
   sp.kpb = s.bk / str; sp.rpq = s.bq / str;
   sp.n_row_tiles = cdiv(sp.nqp, kTileRows);
-  sp.rank = rank; sp.block_score = block_score; sp.hrm_flags = hrm_flags; sp.status = dev_status;
+  sp.rank = rank; sp.bs = bs; sp.block_score = block_score; sp.hrm_flags = hrm_flags; sp.status = dev_status;
   if ((st = launch_status(launch_kap_score(tm_qp, tm_kp, sp, stream))) != COSA_OK) return st;
 
   SortParams so;

@@ -34,6 +34,7 @@ struct ScoreParams {
   int rpq;                      // pooled rows per Q-block (bq / s)
   int n_row_tiles;              // ceil(nqp / 128)
   float* rank;                  // [B, Hq, nQB, nKB] ranking key: +1 for HRM blocks, else score
+  float* bs;                    // [B*Hq, n_row_tiles, nKB, 128] max-pooled block scores, pass 1 -> pass 2
   float* block_score;           // optional [B, Hq, nQB, nKB]
   uint8_t* hrm_flags;           // optional [B, Hq, nQB, nKB]
   uint32_t* status;

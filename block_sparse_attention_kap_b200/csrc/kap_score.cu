@@ -7,14 +7,13 @@
 // accumulators so the next tile's MMA overlaps this tile's epilogue):
 //   S[r, c]   = Qp[r] . Kp[c]                    (raw pooled scores)
 //   Bs[r, j]  = max over visible c in block j     (MaxPool over keys)
-// Pass 1 finds each pooled row's max and the first block attaining it
-// (the HRM block).  Pass 2 recomputes the same tiles (bit-identical) and
-// emits, per (Q-block, KV block), the aggregated MaxNorm score
+// Pass 1 stores Bs to workspace and finds each pooled row's max and the
+// first block attaining it (the HRM block).  Pass 2 reads Bs back (each
+// thread its own values, mostly from L2) and emits, per (Q-block, KV block),
+// the aggregated MaxNorm score
 //   score[I, j] = max over the pooled rows r of I of (Bs[r, j] - rowmax[r])
 // and the HRM flag, packed into one ranking key (+1 for HRM blocks, whose
 // score is 0, else the score <= 0) so the sort needs one array.
-// Recomputing instead of storing Bs keeps the kernel free of a
-// [rows x blocks] scratch buffer; the contraction is cheap next to OSK.
 // Every selection decision (max, subtract, compare) is taken in fp32.
 //
 // Roles: warp 8 issues TMA and MMA; warps 0-7 are the epilogue, two per TMEM
@@ -78,7 +77,7 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
   const int rows_valid = min(kTileRows, p.nqp - r_first);
   const int cmax = p.off_p + r_first + rows_valid - 1;        // last pooled key any row here can see
   const int nT = min(cmax / kTileRows + 1, (p.nkp + kTileRows - 1) / kTileRows);
-  const int U = 2 * nT;
+  const int U = nT;                                            // MMA tiles (pass 1 only)
   constexpr int BPT = kTileRows / KPB;                         // KV blocks per key tile
   constexpr int BPH = BPT / 2;                                 // per 64-column half
 
@@ -160,6 +159,8 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
     const int gl = lane % p.rpq;                // position inside the Q-block's lane group
     float rowmax = -INFINITY;
     int argj = -1;
+    // this row's Bs, [nKB][128 rows] per (head, row tile): coalesced across the warp
+    float* bs_row = p.bs + ((size_t)(b * p.Hq + h) * p.n_row_tiles + R) * p.nkb * kTileRows + row;
     for (int u = 0; u < U; ++u) {
       const int st = u & 1;
       const int T = u % nT;
@@ -190,35 +191,43 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
       tc_fence_before();
       mbar_arrive(&sm->s_free[st]);
       const int j0 = T * BPT + half * BPH;                     // first block of this half
-      if (u < nT) {
 #pragma unroll
-        for (int jh = 0; jh < BPH; ++jh)
-          if (bsv[jh] > rowmax) { rowmax = bsv[jh]; argj = j0 + jh; }
-        if (u == nT - 1) {
-          // merge the two halves: the larger max; on a tie the smaller block index
-          sm->hmax[half][row] = rowmax;
-          sm->harg[half][row] = argj;
-          named_barrier(1, 32 * kEpiWarps);
-          const float m0 = sm->hmax[0][row], m1 = sm->hmax[1][row];
-          const int a0 = sm->harg[0][row], a1 = sm->harg[1][row];
-          rowmax = fmaxf(m0, m1);
-          argj = (m0 > m1) ? a0 : (m1 > m0) ? a1 : min(a0, a1);
-        }
-      } else {
-        // HRM: the Q-block's flags for this half-tile, as a bit mask OR-ed over its rows
-        uint32_t bits = (argj >= j0 && argj < j0 + BPH) ? 1u << (argj - j0) : 0u;
-        for (int o = 1; o < p.rpq; o <<= 1) bits |= __shfl_xor_sync(0xffffffffu, bits, o);
+      for (int jh = 0; jh < BPH; ++jh)
+        if (j0 + jh < p.nkb) bs_row[(size_t)(j0 + jh) * kTileRows] = bsv[jh];
 #pragma unroll
-        for (int jh = 0; jh < BPH; ++jh) {
-          const int j = j0 + jh;
-          float z = (row_ok && bsv[jh] != -INFINITY) ? __fsub_rn(bsv[jh], rowmax) : -INFINITY;
-          for (int o = 1; o < p.rpq; o <<= 1) z = fmaxf(z, __shfl_xor_sync(0xffffffffu, z, o));
-          const uint32_t flag = (bits >> jh) & 1u;
-          if (qblock_ok && (jh % p.rpq) == gl && j < n_I) {
-            p.rank[rank_row + j] = flag ? 1.0f : z;
-            if (p.block_score) p.block_score[rank_row + j] = z;
-            if (p.hrm_flags) p.hrm_flags[rank_row + j] = (uint8_t)flag;
-          }
+      for (int jh = 0; jh < BPH; ++jh)
+        if (bsv[jh] > rowmax) { rowmax = bsv[jh]; argj = j0 + jh; }
+      if (u == nT - 1) {
+        // merge the two halves: the larger max; on a tie the smaller block index
+        sm->hmax[half][row] = rowmax;
+        sm->harg[half][row] = argj;
+        named_barrier(1, 32 * kEpiWarps);
+        const float m0 = sm->hmax[0][row], m1 = sm->hmax[1][row];
+        const int a0 = sm->harg[0][row], a1 = sm->harg[1][row];
+        rowmax = fmaxf(m0, m1);
+        argj = (m0 > m1) ? a0 : (m1 > m0) ? a1 : min(a0, a1);
+      }
+    }
+    // pass 2: MaxNorm, HRM flags and the Q-block aggregate from the stored Bs
+    // (values this thread wrote itself)
+    for (int T = 0; T < nT; ++T) {
+      const int j0 = T * BPT + half * BPH;
+      float bsv[BPH];
+#pragma unroll
+      for (int jh = 0; jh < BPH; ++jh) bsv[jh] = j0 + jh < p.nkb ? bs_row[(size_t)(j0 + jh) * kTileRows] : -INFINITY;
+      // HRM: the Q-block's flags for this half-tile, as a bit mask OR-ed over its rows
+      uint32_t bits = (argj >= j0 && argj < j0 + BPH) ? 1u << (argj - j0) : 0u;
+      for (int o = 1; o < p.rpq; o <<= 1) bits |= __shfl_xor_sync(0xffffffffu, bits, o);
+#pragma unroll
+      for (int jh = 0; jh < BPH; ++jh) {
+        const int j = j0 + jh;
+        float z = (row_ok && bsv[jh] != -INFINITY) ? __fsub_rn(bsv[jh], rowmax) : -INFINITY;
+        for (int o = 1; o < p.rpq; o <<= 1) z = fmaxf(z, __shfl_xor_sync(0xffffffffu, z, o));
+        const uint32_t flag = (bits >> jh) & 1u;
+        if (qblock_ok && (jh % p.rpq) == gl && j < n_I) {
+          p.rank[rank_row + j] = flag ? 1.0f : z;
+          if (p.block_score) p.block_score[rank_row + j] = z;
+          if (p.hrm_flags) p.hrm_flags[rank_row + j] = (uint8_t)flag;
         }
       }
     }

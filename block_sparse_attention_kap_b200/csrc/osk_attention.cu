@@ -256,11 +256,22 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       const bool got = wait_or_abort(&sm->s_full, t & 1, abort, p.status, DEV_TIMEOUT_MMA);
       tc_fence_after();
       const int lim = min(qpos - j * BK, p.Nkv - 1 - j * BK);   // last visible column
-      // pass 1: max over this half's visible columns (TMEM -> registers, 32 at a
-      // time, 4 independent partial maxima)
+      // pass 1: max over this half's visible columns (one 64-column TMEM load
+      // at BK=128, 4 independent partial maxima)
       float mp[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) mp[i] = -INFINITY;
+      if constexpr (HC == 64) {
+        uint32_t v[64];
+        tmem_ld_x64(tS + lane_base + c_base, v);
+        if (lim >= c_base + 63) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) mp[i & 3] = fmaxf(mp[i & 3], __uint_as_float(v[i]));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) mp[i & 3] = fmaxf(mp[i & 3], c_base + i <= lim ? __uint_as_float(v[i]) : -INFINITY);
+        }
+      } else {
 #pragma unroll 1
       for (int c0 = c_base; c0 < c_base + HC; c0 += 32) {
         uint32_t v[32];
@@ -272,6 +283,7 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 #pragma unroll
           for (int i = 0; i < 32; ++i) mp[i & 3] = fmaxf(mp[i & 3], c0 + i <= lim ? __uint_as_float(v[i]) : -INFINITY);
         }
+      }
       }
       const float m_half = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
       const bool vote = !got || !row_ok || !j_ok || m_half == -INFINITY ||

@@ -77,8 +77,9 @@ COSA_API int cosa_num_kblocks(const cosa_shape* shape);
  * cosa_plan.  Returns -1 for an invalid shape or budget outside (0, 1]. */
 COSA_API int cosa_kmax(const cosa_shape* shape, double budget);
 
-/* Bytes of device workspace cosa_plan needs (pooled Q, pooled K and the
- * per-(head, Q-block) block ranking).  0 for an invalid shape. */
+/* Bytes of device workspace cosa_plan needs (pooled Q, pooled K, the
+ * per-(head, Q-block) block ranking and the max-pooled block scores of every
+ * pooled query row).  0 for an invalid shape. */
 COSA_API size_t cosa_plan_workspace_bytes(const cosa_shape* shape);
 
 /* KAP, stage 1 (Sec. 2.2): downsample Q and K (mean of `stride` consecutive
