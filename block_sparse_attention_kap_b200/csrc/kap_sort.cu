@@ -4,22 +4,21 @@
 // and the first k_I = max(1, ceil(n_I * budget)) form the computation-order
 // mask M_KAP.
 //
-// One CTA per (b, h, Q-block).  Each block's ranking key (+1 for HRM blocks,
-// else its score <= 0, written by kap_score) is mapped to an order-preserving
-// 32-bit integer.  A 4-pass, 8-bit radix select finds the k-th largest value
-// T; the blocks above T plus the lowest-indexed blocks equal to T (an ordered
-// block scan) are compacted, and only those k keys -- packed with the
-// inverted block index so ties resolve to the smaller index -- are sorted by
-// a shared-memory bitonic network.  At a 10% budget this sorts a tenth of
-// the keys a full sort would.
+// One warp per (b, h, Q-block), several per CTA, synchronised only with
+// __syncwarp.  Each block's ranking key (+1 for HRM blocks, else its score
+// <= 0, written by kap_score) is mapped to an order-preserving 32-bit
+// integer.  A 4-pass, 8-bit radix select (per-warp shared-memory histogram)
+// finds the k-th largest value T; the blocks above T plus the lowest-indexed
+// blocks equal to T are compacted in index order with warp ballots, and only
+// those k keys -- packed with the inverted block index so ties resolve to
+// the smaller index -- are sorted by a bitonic network in shared memory.
 #include "internal.h"
 
 namespace cosa {
 
 namespace {
 
-constexpr int kSortThreads = 256;
-constexpr int kWarps = kSortThreads / 32;
+constexpr int kMaxWarps = 8;
 
 __device__ __forceinline__ uint32_t orderable(float f) {
   const uint32_t u = __float_as_uint(f);
@@ -31,40 +30,25 @@ __device__ __forceinline__ int causal_blocks(int I, int Nq, int Nkv, int bq, int
   return min(nkb, (Nkv - Nq + last_tok) / bk + 1);
 }
 
-// Exclusive block-wide prefix sum of v (all threads); returns the total too.
-__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) warp_tot[warp] = x;
-  __syncthreads();
-  int base = 0;
-  total = 0;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) {
-    const int t = warp_tot[w];
-    if (w < warp) base += t;
-    total += t;
-  }
-  __syncthreads();
-  return base + x - v;
+__host__ __device__ __forceinline__ size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
+
+// Per-warp shared memory: a 256-bin histogram, the n keys, the P selected keys.
+__host__ __device__ __forceinline__ size_t warp_smem(int nkb, int pk) {
+  return 1024 + align16((size_t)nkb * 4) + (size_t)pk * 8;
 }
 
-__global__ void __launch_bounds__(kSortThreads) kap_sort_kernel(SortParams p, int pmax) {
-  extern __shared__ uint64_t dyn[];
-  uint64_t* sel = dyn;                                          // [pmax] selected keys
-  uint32_t* hi = reinterpret_cast<uint32_t*>(dyn + pmax);        // [pmax] orderable ranking keys
-  __shared__ int hist[256];
-  __shared__ int warp_tot[kWarps];
-  __shared__ uint32_t s_prefix;
-  __shared__ int s_remaining, s_hrm;
+__global__ void __launch_bounds__(32 * kMaxWarps) kap_sort_kernel(SortParams p, int pk, int rows) {
+  extern __shared__ __align__(16) uint8_t dyn[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (row >= rows) return;                       // whole warps only; no block-wide barrier below
+  uint8_t* mine = dyn + (size_t)warp * warp_smem(p.nkb, pk);
+  int* hist = reinterpret_cast<int*>(mine);
+  uint32_t* hi = reinterpret_cast<uint32_t*>(mine + 1024);
+  uint64_t* sel = reinterpret_cast<uint64_t*>(mine + 1024 + align16((size_t)p.nkb * 4));
+  const unsigned full = 0xffffffffu;
+  const unsigned lt_mask = (1u << lane) - 1u;
 
-  const int tid = threadIdx.x;
-  const int row = blockIdx.x;
   const int I = row % p.nqb;
   const int n = causal_blocks(I, p.Nq, p.Nkv, p.bq, p.bk, p.nkb);
   int k = (int)(((long long)n * p.bp + 9999) / 10000);
@@ -72,99 +56,93 @@ __global__ void __launch_bounds__(kSortThreads) kap_sort_kernel(SortParams p, in
   const float* rk = p.rank + (size_t)row * p.nkb;
   const uint32_t hrm_key = orderable(1.0f);
 
-  if (tid == 0) s_hrm = 0;
-  int my_hrm = 0;
-  for (int i = tid; i < n; i += kSortThreads) {
+  int hrm = 0;
+  for (int i = lane; i < n; i += 32) {
     const uint32_t h = orderable(rk[i]);
     hi[i] = h;
-    my_hrm += (h == hrm_key);
+    hrm += (h == hrm_key);
   }
-  __syncthreads();
-  if (my_hrm) atomicAdd(&s_hrm, my_hrm);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) hrm += __shfl_xor_sync(full, hrm, o);
+  __syncwarp();
 
-  // ---------------------------------------------------------------- radix select of the k-th largest
-  uint32_t T = 0;            // threshold value
-  int need = k;              // how many of the elements equal to T are taken
+  // ------------------------------------------------------------ radix select of the k-th largest
+  uint32_t T = 0;
+  int need = k;
   if (k < n) {
     uint32_t prefix = 0, mask = 0;
     int remaining = k;
     for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int b = tid; b < 256; b += kSortThreads) hist[b] = 0;
-      __syncthreads();
-      for (int i = tid; i < n; i += kSortThreads) {
+      for (int b = lane; b < 256; b += 32) hist[b] = 0;
+      __syncwarp();
+      for (int i = lane; i < n; i += 32) {
         const uint32_t h = hi[i];
         if ((h & mask) == prefix) atomicAdd(&hist[(h >> shift) & 255u], 1);
       }
-      __syncthreads();
-      if (tid < 32) {
-        // lane l owns digits 255-8l .. 248-8l (descending); suffix counts from the top digit
-        int c[8], s = 0;
+      __syncwarp();
+      // lane l owns digits 255-8l .. 248-8l (descending); counts from the top digit
+      int c[8], tot = 0;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) { c[q] = hist[255 - 8 * tid - q]; s += c[q]; }
-        int incl = s;
+      for (int q = 0; q < 8; ++q) { c[q] = hist[255 - 8 * lane - q]; tot += c[q]; }
+      int incl = tot;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (tid >= o) incl += y;
-        }
-        const int excl = incl - s;
-        // the lane whose range contains the remaining-th largest element
-        if (excl < remaining && remaining <= incl) {
-          int acc = excl;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(full, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const int excl = incl - tot;
+      const bool here = excl < remaining && remaining <= incl;
+      uint32_t digit = 0;
+      int rem_here = 0;
+      if (here) {
+        int acc = excl;
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            if (acc + c[q] >= remaining) {
-              s_prefix = prefix | ((uint32_t)(255 - 8 * tid - q) << shift);
-              s_remaining = remaining - acc;
-              break;
-            }
-            acc += c[q];
-          }
+        for (int q = 0; q < 8; ++q) {
+          if (acc + c[q] >= remaining) { digit = 255 - 8 * lane - q; rem_here = remaining - acc; break; }
+          acc += c[q];
         }
       }
-      __syncthreads();
-      prefix = s_prefix;
-      remaining = s_remaining;
+      const int src = __ffs(__ballot_sync(full, here)) - 1;
+      digit = __shfl_sync(full, digit, src);
+      remaining = __shfl_sync(full, rem_here, src);
+      prefix |= digit << shift;
       mask |= 255u << shift;
-      __syncthreads();
+      __syncwarp();
     }
     T = prefix;
     need = remaining;
   }
 
-  // ---------------------------------------------------------------- compaction (ordered for ties)
-  const int chunk = (n + kSortThreads - 1) / kSortThreads;
-  const int lo = min(n, tid * chunk), up = min(n, lo + chunk);
-  int gt = 0, eq = 0;
-  if (k < n)
-    for (int i = lo; i < up; ++i) { gt += hi[i] > T; eq += hi[i] == T; }
-  int total_gt, total_eq;
-  const int gt_base = block_exclusive_scan(gt, warp_tot, total_gt);
-  const int eq_base = block_exclusive_scan(eq, warp_tot, total_eq);
-  if (k < n) {
-    int g = gt_base, e = eq_base;
-    for (int i = lo; i < up; ++i) {
-      const uint32_t h = hi[i];
-      const uint64_t key = ((uint64_t)h << 32) | (uint64_t)(0xffffffffu - (uint32_t)i);
-      if (h > T) sel[g++] = key;
-      else if (h == T) {
-        if (e < need) sel[total_gt + e] = key;
-        ++e;
-      }
+  // ------------------------------------------------------------ compaction in index order
+  const int total_gt = k - need;
+  int g = 0, e = 0;
+  for (int base = 0; base < n; base += 32) {
+    const int i = base + lane;
+    const uint32_t h = i < n ? hi[i] : 0u;
+    const uint64_t key = ((uint64_t)h << 32) | (uint64_t)(0xffffffffu - (uint32_t)i);
+    if (k == n) {
+      if (i < n) sel[i] = key;
+      continue;
     }
-  } else {
-    for (int i = lo; i < up; ++i)
-      sel[i] = ((uint64_t)hi[i] << 32) | (uint64_t)(0xffffffffu - (uint32_t)i);
+    const bool gt = i < n && h > T, eq = i < n && h == T;
+    const unsigned bg = __ballot_sync(full, gt), be = __ballot_sync(full, eq);
+    if (gt) sel[g + __popc(bg & lt_mask)] = key;
+    if (eq) {
+      const int r = e + __popc(be & lt_mask);
+      if (r < need) sel[total_gt + r] = key;
+    }
+    g += __popc(bg);
+    e += __popc(be);
   }
   int P = 1;
   while (P < k) P <<= 1;
-  for (int i = k + tid; i < P; i += kSortThreads) sel[i] = 0;
-  __syncthreads();
+  for (int i = k + lane; i < P; i += 32) sel[i] = 0;
+  __syncwarp();
 
-  // ---------------------------------------------------------------- bitonic sort of the k keys, descending
+  // ------------------------------------------------------------ bitonic sort of the k keys, descending
   for (int kk = 2; kk <= P; kk <<= 1) {
     for (int j = kk >> 1; j > 0; j >>= 1) {
-      for (int i = tid; i < P; i += kSortThreads) {
+      for (int i = lane; i < P; i += 32) {
         const int ixj = i ^ j;
         if (ixj > i) {
           const uint64_t a = sel[i], b = sel[ixj];
@@ -175,21 +153,21 @@ __global__ void __launch_bounds__(kSortThreads) kap_sort_kernel(SortParams p, in
           }
         }
       }
-      __syncthreads();
+      __syncwarp();
     }
   }
   int32_t* ord = p.order + (size_t)row * p.kmax;
-  for (int t = tid; t < p.kmax; t += kSortThreads)
+  for (int t = lane; t < p.kmax; t += 32)
     ord[t] = t < k ? (int32_t)(0xffffffffu - (uint32_t)(sel[t] & 0xffffffffu)) : -1;
-  if (tid == 0) {
+  if (lane == 0) {
     p.count[row] = k;
-    if (p.hrm_count) p.hrm_count[row] = s_hrm;
+    if (p.hrm_count) p.hrm_count[row] = hrm;
   }
   // blocks no query of this Q-block can see: -inf score, no flag
   if (p.block_score)
-    for (int j = n + tid; j < p.nkb; j += kSortThreads) p.block_score[(size_t)row * p.nkb + j] = -INFINITY;
+    for (int j = n + lane; j < p.nkb; j += 32) p.block_score[(size_t)row * p.nkb + j] = -INFINITY;
   if (p.hrm_flags)
-    for (int j = n + tid; j < p.nkb; j += kSortThreads) p.hrm_flags[(size_t)row * p.nkb + j] = 0;
+    for (int j = n + lane; j < p.nkb; j += 32) p.hrm_flags[(size_t)row * p.nkb + j] = 0;
 }
 
 __global__ void dense_order_kernel(int rows, int nqb, int nkb, int Nq, int Nkv, int bq, int bk, int kmax,
@@ -205,14 +183,17 @@ __global__ void dense_order_kernel(int rows, int nqb, int nkb, int Nq, int Nkv, 
 cudaError_t launch_kap_sort(const SortParams& p, cudaStream_t st) {
   const int rows = p.B * p.Hq * p.nqb;
   if (rows == 0) return cudaSuccess;
-  int pmax = 1;
-  while (pmax < p.nkb) pmax <<= 1;
-  const size_t smem = (size_t)pmax * (sizeof(uint64_t) + sizeof(uint32_t));
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(kap_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-  }
-  kap_sort_kernel<<<rows, kSortThreads, smem, st>>>(p, pmax);
+  int pk = 1;
+  while (pk < p.kmax) pk <<= 1;
+  const size_t per_warp = warp_smem(p.nkb, pk);
+  int warps = (int)((96 * 1024) / per_warp);
+  warps = warps < 1 ? 1 : (warps > kMaxWarps ? kMaxWarps : warps);
+  const size_t smem = per_warp * warps;
+  if (smem > 227 * 1024) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(kap_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = (unsigned)((rows + warps - 1) / warps);
+  kap_sort_kernel<<<grid, 32 * warps, smem, st>>>(p, pk, rows);
   return cudaGetLastError();
 }
 
