@@ -47,6 +47,19 @@ def lib():
     return _LIB
 
 
+def round_bf16(x: torch.Tensor) -> torch.Tensor:
+    """Round fp64 values to the nearest bf16 value, ties to even, directly
+    from fp64 (no intermediate fp32 rounding), returned as fp64.  The
+    kernels store their fp32 outputs as bf16 with round-to-nearest-even, so
+    this is the closest a bf16 output can be to the exact result."""
+    x = x.double()
+    m, e = torch.frexp(x)                       # x = m * 2^e, 0.5 <= |m| < 1
+    # bf16 keeps 8 significant bits; below 2^-126 the spacing stays 2^-133
+    step = torch.ldexp(torch.ones_like(x), torch.clamp(e - 8, min=-133))
+    r = torch.round(x / step) * step            # torch.round: half to even
+    return torch.where(torch.isfinite(x), r, x)
+
+
 def shape_of(wl) -> OrShape:
     return OrShape(wl.B, wl.Hq, wl.Hkv, wl.Nq, wl.Nkv, wl.d, wl.bq, wl.bk, wl.stride,
                    1 if wl.paged else 0, wl.num_pages)

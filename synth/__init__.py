@@ -27,7 +27,12 @@ available here, so these synthetic inputs stand in for their shapes only):
   blocks.
 * V = z.
 * the integer grid variant draws Q, K, V uniformly from {-2,...,2}; every
-  pooled value and every logit is then exact in bf16 / fp32.
+  pooled value and every logit is then exact in bf16 / fp32.  With structure
+  on, a per-kv-head integer direction w_g in {-1, 0, 1}^d (nonzero on dims
+  0..15) is added as Q += 4 w_g and, on the sink tokens and needle blocks,
+  K += 4 w_g: values stay in {-6..6}, so pooled scores and logits stay exact,
+  while sink and needle logits sit ~200 above the rest and in-kernel skips
+  occur.
 
 All values are rounded to bf16 with round-to-nearest-even (torch's
 float32 -> bfloat16 conversion).  Seeds: 1000 * workload id + tensor id.
@@ -159,6 +164,19 @@ def generate(wl: Workload, grid: bool = False, rank: int = 0) -> Inputs:
         q = torch.randint(-2, 3, (B, Hq, Nq, d), generator=_gen(wid, TENSOR_Q), dtype=torch.int8)
         k = torch.randint(-2, 3, (B, Hkv, Nkv, d), generator=_gen(wid, TENSOR_K), dtype=torch.int8)
         v = torch.randint(-2, 3, (B, Hkv, Nkv, d), generator=_gen(wid, TENSOR_V), dtype=torch.int8)
+        if wl.structured:
+            w = torch.randint(-1, 2, (B, Hkv, d), generator=_gen(wid, TENSOR_DIR), dtype=torch.int8)
+            w[..., 16:] = 0
+            q += 4 * w.repeat_interleave(G, dim=1)[:, :, None, :]
+            k[:, :, :N_SINK_TOKENS] += 4 * w[:, :, None, :]
+            nblk128 = -(-Nkv // 128)
+            gn = _gen(wid, TENSOR_NEEDLE)
+            for b in range(B):
+                for g in range(Hkv):
+                    if wl.n_needle > 0 and nblk128 > 1:
+                        picks = torch.randperm(nblk128 - 1, generator=gn)[: wl.n_needle] + 1
+                        for blk in picks.tolist():
+                            k[b, g, blk * 128:(blk + 1) * 128] += 4 * w[b, g]
         q, k, v = q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
     else:
         q = torch.empty(B, Hq, Nq, d, dtype=torch.bfloat16)

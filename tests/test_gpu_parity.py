@@ -2,8 +2,10 @@
 
 Bar (the benchmark spec): M_KAP (order, count, HRM) and the in-kernel skip
 decisions bit-exact on integer-grid inputs, where every pooled value and
-logit is exact; outputs within max-abs 1e-2 (plus one bf16 half-ulp of the
-value, since |out| >= 4 has a bf16 spacing above 2e-2) and mean-abs 1e-3.
+logit is exact; outputs within max-abs 1e-2 of the exact result (plus one
+bf16 half-ulp of the value, since |out| >= 4 has a bf16 spacing above 2e-2)
+and mean-abs 1e-3 from the exact result rounded to bf16 (the outputs are
+bf16; rounding alone costs ~ulp/4 on average).
 On real-valued inputs the proxy's pooled scores come from tensor-core fp32
 sums, so they are compared with a tolerance derived from fp32 accumulation
 (SCORE_TOL), the GPU's sort is checked exactly against its own scores, and
@@ -71,6 +73,10 @@ def flat(t):
 
 
 def check_out(gpu_rows, ref_rows, extra_atol=None):
+    """Max error against the exact (fp64) oracle output, allowing half a
+    bf16 ulp of the value; mean error against the oracle output rounded to
+    bf16 (nearest even), the closest any bf16 output can be -- on outputs of
+    magnitude ~2 the rounding alone averages ~1.2e-3."""
     g = gpu_rows.double().cpu()
     r = ref_rows.double().cpu()
     err = (g - r).abs()
@@ -78,7 +84,8 @@ def check_out(gpu_rows, ref_rows, extra_atol=None):
     if extra_atol is not None:
         tol = tol + extra_atol
     assert bool((err <= tol).all()), f"max abs err {err.max().item():.4g}"
-    assert err.mean().item() <= MEAN_TOL, f"mean abs err {err.mean().item():.4g}"
+    mean_err = (g - oracle.round_bf16(r)).abs().mean().item()
+    assert mean_err <= MEAN_TOL, f"mean abs err (vs bf16-rounded oracle) {mean_err:.4g}"
     return err.max().item()
 
 
@@ -117,8 +124,9 @@ def _make(shape, grid, structured=False):
 
 @pytest.mark.parametrize("shape", GRID_SHAPES)
 @pytest.mark.parametrize("budget", [0.3, 1.0])
-def test_grid_plan_bit_exact(cosa, shape, budget):
-    inp = _make(shape, grid=True)
+@pytest.mark.parametrize("structured", [False, True])
+def test_grid_plan_bit_exact(cosa, shape, budget, structured):
+    inp = _make(shape, grid=True, structured=structured)
     wl = inp.wl
     _, _, plan = gpu_plan(cosa, inp, budget)
     ref = oracle.kap(inp, budget, want_scores=True)
@@ -133,7 +141,9 @@ def test_grid_plan_bit_exact(cosa, shape, budget):
 @pytest.mark.parametrize("shape", GRID_SHAPES)
 @pytest.mark.parametrize("budget,eps", [(0.5, EPS), (1.0, EPS), (1.0, 0.0)])
 def test_grid_attend_skip_bits_exact(cosa, shape, budget, eps):
-    inp = _make(shape, grid=True)
+    # structured grid: sink and needle logits ~200 above the rest, so blocks
+    # really are skipped in-kernel (every decision >= 0.2 from the threshold)
+    inp = _make(shape, grid=True, structured=True)
     wl = inp.wl
     m, dev, plan = gpu_plan(cosa, inp, budget, scores=False)
     ref_plan = oracle.kap(inp, budget)
@@ -144,6 +154,8 @@ def test_grid_attend_skip_bits_exact(cosa, shape, budget, eps):
     assert torch.equal(bits, ref["skipped"])
     if eps == 0.0:
         assert bits.sum().item() == 0
+    elif budget == 1.0:
+        assert bits.sum().item() > 0          # the skip path is exercised
     check_out(gpu_rows(res["out"], wl), ref["out"])
 
 
@@ -335,3 +347,31 @@ def test_mass_recall_matches_oracle(cosa):
                         oracle.dense(inp)["lse"])
     # each lse is within LSE_TOL of the exact value, so the ratio within ~2*LSE_TOL relative
     assert torch.allclose(rec_gpu, rec_ref, rtol=2 * LSE_TOL, atol=0)
+
+
+EDGE_SHAPES = [
+    dict(Hq=2, Hkv=2, Nq=512, Nkv=512, bq=64, bk=128),                   # small Q-blocks, large KV blocks
+    dict(Hq=2, Hkv=1, Nq=48, Nkv=48, bq=128, bk=128),                    # one partial Q-block and KV block
+    dict(Hq=4, Hkv=4, Nq=80, Nkv=1040, bq=64, bk=64),                    # short chunk, ragged cache, G=1
+    dict(B=2, Hq=4, Hkv=2, Nq=256, Nkv=1280, bq=128, bk=64, paged=True),  # two page tables in one pool
+]
+
+
+@pytest.mark.parametrize("shape", EDGE_SHAPES)
+@pytest.mark.parametrize("budget,eps", [(0.01, EPS), (1.0, 0.5), (0.4, 0.999)])
+def test_edge_shapes_bit_exact(cosa, shape, budget, eps):
+    """Plans and skip decisions bit-exact on grids at the edges: one block per
+    Q-block (1% budget), a threshold that skips nearly everything (eps near 1),
+    partial blocks, G = 1, two batches sharing one page pool."""
+    inp = _make(shape, grid=True, structured=True)
+    wl = inp.wl
+    m, dev, plan = gpu_plan(cosa, inp, budget)
+    ref = oracle.kap(inp, budget, want_scores=True)
+    km = ref["order"].shape[1]
+    assert torch.equal(flat(plan["order"])[:, :km], ref["order"])
+    assert torch.equal(flat(plan["count"]).view(-1), ref["count"])
+    assert torch.equal(flat(plan["block_score"]), ref["score"])
+    res = gpu_attend(m, dev, plan["order"], plan["count"], eps)
+    o = oracle.osk(inp, ref["order"], ref["count"], eps)
+    assert torch.equal(cosa.unpack_skip_bits(flat(res["skip_bits"]), km), o["skipped"])
+    check_out(gpu_rows(res["out"], wl), o["out"])

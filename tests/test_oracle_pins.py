@@ -153,6 +153,26 @@ def test_pool_grid_exact():
     assert torch.equal(p.double(), exact)
 
 
+def test_round_bf16_matches_float_conversion():
+    """Direct fp64 -> bf16 rounding: on fp32-representable values it must
+    agree with the fp32 -> bf16 RNE conversion (no double rounding there);
+    ties go to even; the error never exceeds half a bf16 ulp."""
+    g = torch.Generator().manual_seed(3)
+    x32 = (torch.randn(20000, generator=g) * torch.exp2(torch.randint(-20, 20, (20000,), generator=g).float()))
+    ref = x32.to(torch.bfloat16).double()
+    assert torch.equal(oracle.round_bf16(x32.double()), ref)
+    # exact ties: 1 + 2^-8 sits between 1 and 1 + 2^-7 -> even (1); 1 + 3*2^-8 -> 1 + 2^-6
+    t = torch.tensor([1 + 2 ** -8, 1 + 3 * 2 ** -8, -(2 + 2 ** -7), 0.0, float("inf")], dtype=torch.float64)
+    assert oracle.round_bf16(t).tolist() == [1.0, 1 + 2 ** -6, -2.0, 0.0, float("inf")]
+    # a value just above a tie that fp32 would round onto the tie first
+    y = torch.tensor([1 + 2 ** -8 + 2 ** -40], dtype=torch.float64)
+    assert oracle.round_bf16(y).item() == 1 + 2 ** -7
+    z = torch.randn(5000, generator=g, dtype=torch.float64) * 3
+    err = (oracle.round_bf16(z) - z).abs()
+    half_ulp = torch.ldexp(torch.ones_like(z), torch.frexp(z)[1] - 9)
+    assert bool((err <= half_ulp).all())
+
+
 def test_pool_normal_within_half_ulp():
     g = torch.Generator().manual_seed(6)
     x = torch.randn(4096, 64, generator=g).to(torch.bfloat16)
@@ -388,10 +408,10 @@ def test_skip_error_bound_and_monotone():
 def test_skip_decisions_bruteforce_grid():
     """On integer grids every logit is an exact integer: recompute each skip
     decision from the definition with numpy integers."""
-    wl = tiny(Hq=2, Hkv=1, Nq=256, Nkv=256, bq=64, bk=64, d=16)
+    wl = tiny(Hq=2, Hkv=1, Nq=512, Nkv=512, bq=64, bk=64, d=32, structured=True, n_needle=2)
     inp = synth.generate(wl, grid=True)
     plan = oracle.kap(inp, 1.0)
-    eps = 0.05
+    eps = 1e-3
     T = math.log(eps) * math.sqrt(wl.d)
     res = oracle.osk(inp, plan["order"], plan["count"], eps)
     q = inp.q.long().numpy()
@@ -413,6 +433,7 @@ def test_skip_decisions_bruteforce_grid():
                 assert res["skipped"][i, t].item() == int(skip)
                 if not skip:
                     m_run = np.maximum(m_run, m_loc)
+    assert res["skipped"].sum().item() > 0          # decisions of both kinds were checked
 
 
 # ----------------------------------------------------------------- attention-mass recall of M_KAP
