@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--budget B] [--eps E] [--impl cosa|reference]
+                    [--sweep | --chunked]
 
 One step = one pass of the whole hot path over one batch of synthetic
 input: cosa_plan (kap_pool, kap_score, kap_sort) then cosa_attend
@@ -46,12 +47,18 @@ def parse():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="gqa_128k", choices=list(synth.WORKLOADS))
+    ap.add_argument("--heads", default=None, metavar="HQ:HKV",
+                    help="override the workload's query/kv head counts (a smaller case of the same layer, "
+                         "e.g. for profiling); the workload is then reported as NAME[hqHQ:hkvHKV]")
     ap.add_argument("--budget", type=float, default=None)
     ap.add_argument("--eps", type=float, default=None)
     ap.add_argument("--impl", default="cosa", choices=["cosa", "reference"])
     ap.add_argument("--no-dense", action="store_true", help="skip timing the dense path")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
+    ap.add_argument("--chunked", action="store_true",
+                    help="chunked prefill: KAP with the pooled keys kept across chunks (cosa_plan_chunk) "
+                         "against KAP that re-pools the whole cache (cosa_plan), one line (no headline line)")
     ap.add_argument("--sweep", action="store_true",
                     help="one line per budget of the workload: latency, in-kernel skip fraction and error "
                          "against the dense path (no headline line)")
@@ -273,11 +280,104 @@ def run_sweep(args, wl, eps):
                             "min": recall.min().item()}}), flush=True)
 
 
+# ----------------------------------------------------------------- chunked prefill
+
+def run_chunked(args, wl, budget, eps):
+    """One prefill chunk (Nq new queries after Nkv - Nq cached keys): plan
+    latency when every key is pooled again (cosa_plan) and when the pooled
+    keys of earlier chunks come from a cache (cosa_plan_chunk), the attend
+    latency on that plan, and the block union of the plan over the chunk's
+    Q-blocks and each group's heads (CompactAttention's selection stage)
+    executed with eps 0 and with in-kernel skipping; errors against the
+    dense path."""
+    import block_sparse_attention_kap_b200 as cosa
+    if wl.Nkv == wl.Nq:
+        raise SystemExit("--chunked needs a workload with cached keys (Nkv > Nq)")
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    inp = synth.generate(wl)
+    q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
+    pt = inp.page_table.to(dev) if inp.page_table is not None else None
+    shape = cosa.shape_of_workload(wl)
+    m = cosa.CoSA(shape, device=dev)
+    order, count, hrm = m.alloc_plan(budget)
+    km = order.shape[-1]
+    nkp, valid = wl.Nkv // wl.stride, (wl.Nkv - wl.Nq) // wl.stride
+    cache = torch.empty(wl.B, wl.Hkv, nkp, wl.d, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(wl.B, wl.Hq, wl.Nq, wl.d, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    ws = m.workspace()
+    cosa.cosa_plan_chunk(shape, q, k, pt, cache, 0, budget, km, order, count, hrm, None, None, ws, m.status,
+                         stream)
+
+    def timed(fn):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / args.steps
+
+    full_ms = timed(lambda: cosa.cosa_plan(shape, q, k, pt, budget, km, order, count, hrm, None, None, ws,
+                                           m.status, stream))
+    full_order = order.clone()
+    chunk_ms = timed(lambda: cosa.cosa_plan_chunk(shape, q, k, pt, cache, valid, budget, km, order, count, hrm,
+                                                  None, None, ws, m.status, stream))
+    attend_ms = timed(lambda: cosa.cosa_attend(shape, q, k, v, pt, order, count, km, eps, out, None, None,
+                                               m.status, stream))
+    # block union of the plan (per kv-head group, over the chunk's Q-blocks and
+    # the group's heads), executed densely (eps 0) and with in-kernel skipping
+    ures = m.block_union(order, count)
+    u_order, u_count = ures["order"], ures["count"]
+    u_km = u_order.shape[-1]
+    union_ms = timed(lambda: cosa.cosa_block_union(shape, order, count, km, ures["table"], ures["table_len"],
+                                                   u_order, u_count, stream))
+    out_u = torch.empty_like(out)
+    attend_union_dense_ms = timed(lambda: cosa.cosa_attend(shape, q, k, v, pt, u_order, u_count, u_km, 0.0, out_u,
+                                                           None, None, m.status, stream))
+    attend_union_eps_ms = timed(lambda: cosa.cosa_attend(shape, q, k, v, pt, u_order, u_count, u_km, eps, out_u,
+                                                         None, None, m.status, stream))
+    torch.cuda.synchronize()
+    assert m.device_status() == 0
+    assert torch.equal(order, full_order), "cached pooled keys changed the plan"
+    # errors against the dense path on the same inputs
+    dense_out = m.dense(q, k, v, page_table=pt)["out"].float()
+    kap_out = m.attend(q, k, v, order, count, eps, page_table=pt)["out"].float()
+    union_dense_out = m.attend(q, k, v, u_order, u_count, 0.0, page_table=pt)["out"].float()
+    torch.cuda.synchronize()
+    err = lambda o: {"max_abs": (o - dense_out).abs().max().item(), "mean_abs": (o - dense_out).abs().mean().item()}
+    union_blocks = int(u_count.sum().item())
+    kap_blocks = int(count.sum().item())
+    row = 2.0 * wl.d
+    q_bytes = row * wl.B * wl.Hq * wl.Nq * (1 + 1 / wl.stride)
+    full_bytes = q_bytes + row * wl.B * wl.Hkv * wl.Nkv * (1 + 1 / wl.stride)
+    chunk_bytes = q_bytes + row * wl.B * wl.Hkv * (wl.Nq * (1 + 1 / wl.stride) + wl.Nkv / wl.stride)
+    print(json.dumps({
+        "kind": "chunked", "workload": wl.name, "budget": budget, "eps": eps, "Nq": wl.Nq, "Nkv": wl.Nkv,
+        "plan_full_ms": full_ms, "plan_chunk_ms": chunk_ms, "plan_speedup": full_ms / chunk_ms,
+        "attend_ms": attend_ms, "step_full_ms": full_ms + attend_ms, "step_chunk_ms": chunk_ms + attend_ms,
+        "kap_blocks": kap_blocks, "err_kap_vs_dense": err(kap_out),
+        "union": {"union_ms": union_ms, "blocks": union_blocks, "attend_eps0_ms": attend_union_dense_ms,
+                  "attend_eps_ms": attend_union_eps_ms,
+                  "step_eps0_ms": chunk_ms + union_ms + attend_union_dense_ms,
+                  "err_eps0_vs_dense": err(union_dense_out)},
+        "pool_bytes": {"full": full_bytes, "chunk": chunk_bytes},
+        "dense_causal_tflop": wl.dense_causal_flops() / 1e12,
+        "effective_tflops_chunk": wl.dense_causal_flops() / ((chunk_ms + attend_ms) * 1e-3) / 1e12}), flush=True)
+
+
 # ----------------------------------------------------------------- GPU arm
 
 def main():
     args = parse()
     wl = synth.WORKLOADS[args.workload]
+    if args.heads:
+        hq, hkv = (int(x) for x in args.heads.split(":"))
+        wl = wl.replace(Hq=hq, Hkv=hkv, name=f"{wl.name}[hq{hq}:hkv{hkv}]")
     budget = args.budget if args.budget is not None else (0.1 if 0.1 in wl.budgets else wl.budgets[0])
     eps = args.eps if args.eps is not None else wl.eps
     if args.impl == "reference":
@@ -285,6 +385,9 @@ def main():
         return
     if args.sweep:
         run_sweep(args, wl, eps)
+        return
+    if args.chunked:
+        run_chunked(args, wl, budget, eps)
         return
     if args.warmup < 3:
         args.warmup = 3

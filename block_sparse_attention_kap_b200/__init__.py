@@ -54,7 +54,10 @@ _lib.cosa_plan_workspace_bytes.argtypes = [_S]
 _lib.cosa_plan_workspace_bytes.restype = ctypes.c_size_t
 _lib.cosa_plan.argtypes = [_S, _P, _P, _P, ctypes.c_double, ctypes.c_int, _P, _P, _P, _P, _P, _P,
                            ctypes.c_size_t, _P, _P]
+_lib.cosa_plan_chunk.argtypes = [_S, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
+                                 _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]
 _lib.cosa_dense_order.argtypes = [_S, ctypes.c_int, _P, _P, _P]
+_lib.cosa_block_union.argtypes = [_S, _P, _P, ctypes.c_int, _P, _P, _P, _P, ctypes.c_int, _P]
 _lib.cosa_plan_static.argtypes = [_S, _P, _P, _P, ctypes.c_double, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P]
 _lib.cosa_attend.argtypes = [_S, _P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_double, _P, _P, _P, _P, _P]
 _lib.cosa_skip_threshold.argtypes = [ctypes.c_double, ctypes.c_int]
@@ -64,7 +67,7 @@ _lib.cosa_status_string.restype = ctypes.c_char_p
 
 EXPORTS = ("cosa_num_qblocks", "cosa_num_kblocks", "cosa_kmax", "cosa_plan_workspace_bytes", "cosa_plan",
            "cosa_dense_order", "cosa_attend", "cosa_skip_threshold", "cosa_status_string", "cosa_version",
-           "cosa_plan_static")
+           "cosa_plan_static", "cosa_plan_chunk", "cosa_block_union")
 STATIC_SCRATCH_BYTES = 64 << 20
 
 
@@ -137,6 +140,26 @@ def cosa_plan(shape: cosa_shape, q, k, page_table, budget: float, kmax: int, ord
                           _ptr(dev_status, "dev_status", torch.int32), _stream(stream)), "cosa_plan")
 
 
+def cosa_plan_chunk(shape: cosa_shape, q, k, page_table, kp_cache, kp_valid: int, budget: float, kmax: int,
+                    order, count, hrm_count=None, block_score=None, hrm_flags=None, workspace=None,
+                    dev_status=None, stream=None) -> None:
+    """cosa_plan for one prefill chunk: kp_cache [B, Hkv, capacity, d] bf16
+    keeps the pooled keys across chunks; its rows below kp_valid are reused,
+    the rest are pooled from k and written back."""
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    if kp_cache is not None and kp_cache.dim() != 4:
+        raise ValueError("kp_cache must be [B, Hkv, capacity, d]")
+    cap = kp_cache.shape[2] if kp_cache is not None else 0
+    _check(_lib.cosa_plan_chunk(ctypes.byref(shape), _ptr(q, "q", torch.bfloat16), _ptr(k, "k", torch.bfloat16),
+                                _ptr(page_table, "page_table", torch.int32),
+                                _ptr(kp_cache, "kp_cache", torch.bfloat16), cap, kp_valid, budget, kmax,
+                                _ptr(order, "order", torch.int32), _ptr(count, "count", torch.int32),
+                                _ptr(hrm_count, "hrm_count", torch.int32),
+                                _ptr(block_score, "block_score", torch.float32),
+                                _ptr(hrm_flags, "hrm_flags", torch.uint8), _ptr(workspace, "workspace"), ws_bytes,
+                                _ptr(dev_status, "dev_status", torch.int32), _stream(stream)), "cosa_plan_chunk")
+
+
 def cosa_plan_static(shape: cosa_shape, q, k, page_table, budget: float, kmax: int, order, count,
                      hrm_count=None, block_score=None, hrm_flags=None, dev_status=None, stream=None) -> None:
     """cosa_plan for callers that cannot supply a workspace: the scratch is a
@@ -154,6 +177,17 @@ def cosa_plan_static(shape: cosa_shape, q, k, page_table, budget: float, kmax: i
 def cosa_dense_order(shape: cosa_shape, kmax: int, order, count, stream=None) -> None:
     _check(_lib.cosa_dense_order(ctypes.byref(shape), kmax, _ptr(order, "order", torch.int32),
                                  _ptr(count, "count", torch.int32), _stream(stream)), "cosa_dense_order")
+
+
+def cosa_block_union(shape: cosa_shape, order, count, kmax: int, table, table_len, union_order=None,
+                     union_count=None, stream=None) -> None:
+    union_kmax = union_order.shape[-1] if union_order is not None else 0
+    _check(_lib.cosa_block_union(ctypes.byref(shape), _ptr(order, "order", torch.int32),
+                                 _ptr(count, "count", torch.int32), kmax, _ptr(table, "table", torch.int32),
+                                 _ptr(table_len, "table_len", torch.int32),
+                                 _ptr(union_order, "union_order", torch.int32),
+                                 _ptr(union_count, "union_count", torch.int32), union_kmax, _stream(stream)),
+           "cosa_block_union")
 
 
 def cosa_attend(shape: cosa_shape, q, k, v, page_table, order, count, kmax: int, skip_eps: float, out,
@@ -215,6 +249,37 @@ class CoSA:
         if scores:
             res.update(block_score=bs, hrm=hf)
         return res
+
+    def plan_chunk(self, q, k, budget: float, kp_cache, kp_valid: int, page_table=None, out=None,
+                   scores: bool = False, stream=None):
+        """plan() for one chunk of a chunked prefill, reusing the pooled keys
+        kept in kp_cache (rows below kp_valid) and pooling only the rest."""
+        order, count, hrm = out if out is not None else self.alloc_plan(budget)
+        bs = hf = None
+        if scores:
+            s = self.shape
+            bs = torch.empty(s.B, s.Hq, self.nqb, self.nkb, dtype=torch.float32, device=self.device)
+            hf = torch.empty(s.B, s.Hq, self.nqb, self.nkb, dtype=torch.uint8, device=self.device)
+        cosa_plan_chunk(self.shape, q, k, page_table, kp_cache, kp_valid, budget, order.shape[-1], order, count,
+                        hrm, bs, hf, self.workspace(), self.status, stream)
+        res = dict(order=order, count=count, hrm_count=hrm)
+        if scores:
+            res.update(block_score=bs, hrm=hf)
+        return res
+
+    def block_union(self, order, count, expand: bool = True, stream=None):
+        """Per-(batch, kv-head) union of a selection over the Q-blocks and the
+        heads of each group; with expand, also the causally visible prefix
+        of the table per Q-block as an order for attend()."""
+        s = self.shape
+        table = torch.empty(s.B, s.Hkv, self.nkb, dtype=torch.int32, device=self.device)
+        table_len = torch.empty(s.B, s.Hkv, dtype=torch.int32, device=self.device)
+        uo = uc = None
+        if expand:
+            uo = torch.empty(s.B, s.Hq, self.nqb, self.nkb, dtype=torch.int32, device=self.device)
+            uc = torch.empty(s.B, s.Hq, self.nqb, dtype=torch.int32, device=self.device)
+        cosa_block_union(s, order, count, order.shape[-1], table, table_len, uo, uc, stream)
+        return dict(table=table, table_len=table_len, order=uo, count=uc)
 
     def dense_order(self, stream=None):
         s = self.shape

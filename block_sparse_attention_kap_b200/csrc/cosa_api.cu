@@ -9,6 +9,7 @@
 
 #include "cosa.h"
 #include "internal.h"
+#include "block_union.h"
 
 using namespace cosa;
 
@@ -93,24 +94,127 @@ int budget_k(int n, int bp) {
   return (int)k;
 }
 
+// Work items per row tile of kap_score (S): enough CTAs to fill the GPU
+// (four per CTA slot, two slots per SM), no item longer than an eighth of a
+// slot's share of all key tiles (so the longest rows leave no tail), and at
+// least four key tiles per item where rows are long enough (a CTA's set-up
+// is worth a few tiles).
+int score_splits(const cosa_shape* s) {
+  const int nqp = s->Nq / s->stride, nkp = s->Nkv / s->stride, off_p = (s->Nkv - s->Nq) / s->stride;
+  const int nrt = cdiv(nqp, kTileRows);
+  if (nrt == 0 || s->B == 0) return 1;
+  long long tiles = 0;
+  int nt_max = 0;
+  for (int R = 0; R < nrt; ++R) {
+    const int nt = kap_row_tiles_seen(R, nqp, nkp, off_p);
+    tiles += nt;
+    nt_max = std::max(nt_max, nt);
+  }
+  const long long heads = (long long)s->B * s->Hq, slots = 2ll * 148;
+  tiles *= heads;
+  const long long s_fill = (4 * slots + heads * nrt - 1) / (heads * nrt);
+  const long long s_tail = (8ll * nt_max * slots + tiles - 1) / std::max(1ll, tiles);
+  const long long s_cap = std::max(1, nt_max / 4);
+  return (int)std::max(1ll, std::min(std::max(s_fill, s_tail), s_cap));
+}
+
 struct Workspace {
-  size_t qp, kp, rank, bs, total;
+  size_t qp, kp, bs, pmax, parg, total;
+  int splits;
 };
 
 Workspace carve(const cosa_shape* s) {
   Workspace w;
   const long long rows_q = std::max<long long>((long long)s->B * s->Hq * (s->Nq / s->stride), 0) + 128;
   const long long rows_k = std::max<long long>((long long)s->B * s->Hkv * (s->Nkv / s->stride), 0) + 128;
+  const size_t row_tiles = (size_t)cdiv(s->Nq / s->stride, kTileRows);
+  const size_t heads = (size_t)s->B * s->Hq;
+  w.splits = score_splits(s);
   w.qp = 0;
   w.kp = align256(w.qp + (size_t)rows_q * kD * 2);
-  w.rank = align256(w.kp + (size_t)rows_k * kD * 2);
-  w.bs = align256(w.rank + (size_t)s->B * s->Hq * n_qblocks(s) * n_kblocks(s) * sizeof(float));
-  const size_t row_tiles = (size_t)cdiv(s->Nq / s->stride, kTileRows);
-  w.total = align256(w.bs + (size_t)s->B * s->Hq * row_tiles * n_kblocks(s) * kTileRows * sizeof(float));
+  w.bs = align256(w.kp + (size_t)rows_k * kD * 2);
+  w.pmax = align256(w.bs + heads * row_tiles * n_kblocks(s) * kTileRows * sizeof(float));
+  w.parg = align256(w.pmax + heads * row_tiles * w.splits * 2 * kTileRows * sizeof(float));
+  w.total = align256(w.parg + heads * row_tiles * w.splits * 2 * kTileRows * sizeof(int32_t));
   return w;
 }
 
 cosa_status launch_status(cudaError_t e) { return e == cudaSuccess ? COSA_OK : COSA_ECUDA; }
+
+// Shared body of cosa_plan and cosa_plan_chunk.  Pooled keys live in `kp`
+// ([B, Hkv, kp_stride, d]); rows kp_first .. Nkv/s-1 are pooled from k here,
+// rows below kp_first are read as they are.
+cosa_status plan_impl(const cosa_shape* shape, const void* q, const void* k, const int32_t* page_table,
+                      uint16_t* kp, long long kp_map_rows, int kp_stride, int kp_first, double budget,
+                      int kmax, int32_t* order, int32_t* count, int32_t* hrm_count, float* block_score,
+                      uint8_t* hrm_flags, uint8_t* ws, uint32_t* dev_status, cudaStream_t stream) {
+  cosa_status st;
+  const cosa_shape& s = *shape;
+  const Workspace w = carve(&s);
+  uint16_t* qp = reinterpret_cast<uint16_t*>(ws + w.qp);
+  float* bs = reinterpret_cast<float*>(ws + w.bs);
+  float* pmax = reinterpret_cast<float*>(ws + w.pmax);
+  int32_t* parg = reinterpret_cast<int32_t*>(ws + w.parg);
+  const int str = s.stride;
+
+  PoolParams pp;
+  pp.q = static_cast<const uint16_t*>(q);
+  pp.k = static_cast<const uint16_t*>(k);
+  pp.page_table = page_table;
+  pp.qp = qp;
+  pp.kp = kp;
+  pp.B = s.B; pp.Hq = s.Hq; pp.Hkv = s.Hkv; pp.Nq = s.Nq; pp.Nkv = s.Nkv; pp.s = str; pp.bk = s.bk;
+  pp.nkb = n_kblocks(&s); pp.paged = s.paged; pp.num_pages = s.num_pages;
+  pp.kp_first = kp_first; pp.kp_stride = kp_stride;
+  pp.q_items = (long long)s.B * s.Hq * (s.Nq / str);
+  pp.k_items = (long long)s.B * s.Hkv * (s.Nkv / str - kp_first);
+  if ((st = launch_status(launch_kap_pool(pp, stream))) != COSA_OK) return st;
+
+  CUtensorMap tm_qp, tm_kp;
+  if ((st = make_map(&tm_qp, qp, pp.q_items + 128, 128)) != COSA_OK) return st;
+  if ((st = make_map(&tm_kp, kp, kp_map_rows, 128)) != COSA_OK) return st;
+  ScoreParams sp;
+  sp.B = s.B; sp.Hq = s.Hq; sp.Hkv = s.Hkv; sp.G = s.Hq / s.Hkv;
+  sp.nqp = s.Nq / str; sp.nkp = s.Nkv / str; sp.kp_stride = kp_stride; sp.off_p = (s.Nkv - s.Nq) / str;
+  sp.nkb = n_kblocks(&s);
+  sp.kpb = s.bk / str;
+  sp.n_row_tiles = cdiv(sp.nqp, kTileRows);
+  sp.splits = w.splits;
+  sp.bs = bs; sp.part_max = pmax; sp.part_arg = parg; sp.status = dev_status;
+  if ((st = launch_status(launch_kap_score(tm_qp, tm_kp, sp, stream))) != COSA_OK) return st;
+
+  SortParams so;
+  so.B = s.B; so.Hq = s.Hq; so.nqb = n_qblocks(&s); so.nkb = sp.nkb; so.Nq = s.Nq; so.Nkv = s.Nkv;
+  so.bq = s.bq; so.bk = s.bk; so.rpq = s.bq / str;
+  so.nqp = sp.nqp; so.n_row_tiles = sp.n_row_tiles; so.splits = sp.splits;
+  so.bp = budget_bp(budget); so.kmax = kmax;
+  so.bs = bs; so.part_max = pmax; so.part_arg = parg;
+  so.order = order; so.count = count; so.hrm_count = hrm_count;
+  so.block_score = block_score; so.hrm_flags = hrm_flags;
+  return launch_status(launch_kap_sort(so, stream));
+}
+
+// Checks common to cosa_plan and cosa_plan_chunk.  *done is set when there
+// is nothing to launch (no Q-blocks).
+cosa_status check_plan_args(const cosa_shape* shape, const void* q, const void* k,
+                            const int32_t* page_table, double budget, int kmax, const int32_t* order,
+                            const int32_t* count, const void* workspace, size_t ws_bytes, bool* done) {
+  *done = false;
+  cosa_status st = check_plan_shape(shape);
+  if (st != COSA_OK) return st;
+  if (!(budget > 0.0) || budget > 1.0) return COSA_EINVAL;
+  const cosa_shape& s = *shape;
+  if ((long long)s.B * s.Hq * n_qblocks(&s) == 0) {
+    *done = true;
+    return COSA_OK;
+  }
+  if (!q || !k || !order || !count || (s.paged && !page_table)) return COSA_EINVAL;
+  if (!aligned16(q) || !aligned16(k)) return COSA_EALIGN;
+  if (kmax < cosa_kmax(&s, budget)) return COSA_EINVAL;
+  if (!workspace || ws_bytes < carve(&s).total) return COSA_EWORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255) return COSA_EALIGN;
+  return COSA_OK;
+}
 
 }  // namespace
 
@@ -139,56 +243,35 @@ cosa_status cosa_plan(const cosa_shape* shape, const void* q, const void* k, con
                       double budget, int kmax, int32_t* order, int32_t* count, int32_t* hrm_count,
                       float* block_score, uint8_t* hrm_flags, void* workspace, size_t ws_bytes,
                       uint32_t* dev_status, cudaStream_t stream) {
-  cosa_status st = check_plan_shape(shape);
-  if (st != COSA_OK) return st;
-  if (!(budget > 0.0) || budget > 1.0) return COSA_EINVAL;
+  bool done;
+  cosa_status st = check_plan_args(shape, q, k, page_table, budget, kmax, order, count, workspace, ws_bytes, &done);
+  if (st != COSA_OK || done) return st;
   const cosa_shape& s = *shape;
-  const long long rows = (long long)s.B * s.Hq * n_qblocks(&s);
-  if (rows == 0) return COSA_OK;
-  if (!q || !k || !order || !count || (s.paged && !page_table)) return COSA_EINVAL;
-  if (!aligned16(q) || !aligned16(k)) return COSA_EALIGN;
-  if (kmax < cosa_kmax(&s, budget)) return COSA_EINVAL;
-  const Workspace w = carve(&s);
-  if (!workspace || ws_bytes < w.total) return COSA_EWORKSPACE;
-  if (reinterpret_cast<uintptr_t>(workspace) & 255) return COSA_EALIGN;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  uint16_t* qp = reinterpret_cast<uint16_t*>(ws + w.qp);
-  uint16_t* kp = reinterpret_cast<uint16_t*>(ws + w.kp);
-  float* rank = reinterpret_cast<float*>(ws + w.rank);
-  float* bs = reinterpret_cast<float*>(ws + w.bs);
-  const int str = s.stride;
+  const Workspace w = carve(&s);
+  const int nkp = s.Nkv / s.stride;
+  return plan_impl(&s, q, k, page_table, reinterpret_cast<uint16_t*>(ws + w.kp),
+                   (long long)s.B * s.Hkv * nkp + 128, nkp, 0, budget, kmax, order, count, hrm_count,
+                   block_score, hrm_flags, ws, dev_status, stream);
+}
 
-  PoolParams pp;
-  pp.q = static_cast<const uint16_t*>(q);
-  pp.k = static_cast<const uint16_t*>(k);
-  pp.page_table = page_table;
-  pp.qp = qp;
-  pp.kp = kp;
-  pp.B = s.B; pp.Hq = s.Hq; pp.Hkv = s.Hkv; pp.Nq = s.Nq; pp.Nkv = s.Nkv; pp.s = str; pp.bk = s.bk;
-  pp.nkb = n_kblocks(&s); pp.paged = s.paged; pp.num_pages = s.num_pages;
-  pp.q_items = (long long)s.B * s.Hq * (s.Nq / str);
-  pp.k_items = (long long)s.B * s.Hkv * (s.Nkv / str);
-  if ((st = launch_status(launch_kap_pool(pp, stream))) != COSA_OK) return st;
-
-  CUtensorMap tm_qp, tm_kp;
-  if ((st = make_map(&tm_qp, qp, pp.q_items + 128, 128)) != COSA_OK) return st;
-  if ((st = make_map(&tm_kp, kp, pp.k_items + 128, 128)) != COSA_OK) return st;
-  ScoreParams sp;
-  sp.B = s.B; sp.Hq = s.Hq; sp.Hkv = s.Hkv; sp.G = s.Hq / s.Hkv;
-  sp.nqp = s.Nq / str; sp.nkp = s.Nkv / str; sp.off_p = (s.Nkv - s.Nq) / str;
-  sp.Nq = s.Nq; sp.Nkv = s.Nkv; sp.bq = s.bq; sp.bk = s.bk; sp.s = str;
-  sp.nqb = n_qblocks(&s); sp.nkb = n_kblocks(&s);
-  sp.kpb = s.bk / str; sp.rpq = s.bq / str;
-  sp.n_row_tiles = cdiv(sp.nqp, kTileRows);
-  sp.rank = rank; sp.bs = bs; sp.block_score = block_score; sp.hrm_flags = hrm_flags; sp.status = dev_status;
-  if ((st = launch_status(launch_kap_score(tm_qp, tm_kp, sp, stream))) != COSA_OK) return st;
-
-  SortParams so;
-  so.B = s.B; so.Hq = s.Hq; so.nqb = sp.nqb; so.nkb = sp.nkb; so.Nq = s.Nq; so.Nkv = s.Nkv;
-  so.bq = s.bq; so.bk = s.bk; so.bp = budget_bp(budget); so.kmax = kmax;
-  so.rank = rank; so.order = order; so.count = count; so.hrm_count = hrm_count;
-  so.block_score = block_score; so.hrm_flags = hrm_flags;
-  return launch_status(launch_kap_sort(so, stream));
+cosa_status cosa_plan_chunk(const cosa_shape* shape, const void* q, const void* k, const int32_t* page_table,
+                            void* kp_cache, int kp_capacity, int kp_valid, double budget, int kmax,
+                            int32_t* order, int32_t* count, int32_t* hrm_count, float* block_score,
+                            uint8_t* hrm_flags, void* workspace, size_t ws_bytes, uint32_t* dev_status,
+                            cudaStream_t stream) {
+  bool done;
+  cosa_status st = check_plan_args(shape, q, k, page_table, budget, kmax, order, count, workspace, ws_bytes, &done);
+  if (st != COSA_OK || done) return st;
+  const cosa_shape& s = *shape;
+  const int nkp = s.Nkv / s.stride;
+  if (!kp_cache) return COSA_EINVAL;
+  if (!aligned16(kp_cache)) return COSA_EALIGN;
+  if (kp_capacity < nkp || kp_valid < 0 || kp_valid > nkp) return COSA_EINVAL;
+  if ((long long)s.B * s.Hkv * kp_capacity >= (1ll << 31)) return COSA_EUNSUPPORTED;
+  return plan_impl(&s, q, k, page_table, static_cast<uint16_t*>(kp_cache), (long long)s.B * s.Hkv * kp_capacity,
+                   kp_capacity, kp_valid, budget, kmax, order, count, hrm_count, block_score, hrm_flags,
+                   static_cast<uint8_t*>(workspace), dev_status, stream);
 }
 
 cosa_status cosa_dense_order(const cosa_shape* shape, int kmax, int32_t* order, int32_t* count,
@@ -201,6 +284,29 @@ cosa_status cosa_dense_order(const cosa_shape* shape, int kmax, int32_t* order, 
   if (kmax < causal_blocks(shape, n_qblocks(shape) - 1)) return COSA_EINVAL;
   return launch_status(launch_dense_order(rows, n_qblocks(shape), n_kblocks(shape), shape->Nq, shape->Nkv,
                                           shape->bq, shape->bk, kmax, order, count, stream));
+}
+
+cosa_status cosa_block_union(const cosa_shape* shape, const int32_t* order, const int32_t* count, int kmax,
+                             int32_t* table, int32_t* table_len, int32_t* union_order, int32_t* union_count,
+                             int union_kmax, cudaStream_t stream) {
+  cosa_status st = check_shape(shape);
+  if (st != COSA_OK) return st;
+  const cosa_shape& s = *shape;
+  if ((long long)s.B * s.Hkv == 0) return COSA_OK;
+  if (!table || !table_len || kmax < 0) return COSA_EINVAL;
+  const int nqb = n_qblocks(&s);
+  if (nqb > 0 && kmax > 0 && (!order || !count)) return COSA_EINVAL;
+  if (union_order || union_count) {
+    if (!union_order || !union_count) return COSA_EINVAL;
+    if (nqb > 0 && union_kmax < causal_blocks(&s, nqb - 1)) return COSA_EINVAL;
+  }
+  UnionParams p;
+  p.B = s.B; p.Hq = s.Hq; p.Hkv = s.Hkv; p.nqb = nqb; p.nkb = n_kblocks(&s);
+  p.Nq = s.Nq; p.Nkv = s.Nkv; p.bq = s.bq; p.bk = s.bk;
+  p.order = order; p.count = count; p.kmax = (nqb > 0) ? kmax : 0;
+  p.table = table; p.table_len = table_len;
+  p.union_order = union_order; p.union_count = union_count; p.union_kmax = union_kmax;
+  return launch_status(launch_block_union(p, stream));
 }
 
 cosa_status cosa_attend(const cosa_shape* shape, const void* q, const void* k, const void* v,
@@ -246,6 +352,6 @@ const char* cosa_status_string(cosa_status status) {
   return "COSA: unknown status";
 }
 
-int cosa_version(void) { return 100; }
+int cosa_version(void) { return 101; }
 
 }  // extern "C"

@@ -62,14 +62,16 @@ __global__ void __launch_bounds__(256) kap_pool_kernel(PoolParams p) {
     src = p.q + item * s * kD;   // pooled row item of head (b,h) starts at token item*s of the flat Q
     dst = p.qp + item * kD;
   } else {
+    // K rows kp_first .. Nkv/s-1 of each (b, kv-head); rows below kp_first
+    // were pooled by an earlier call (chunked prefill) and are not touched
+    const int n_new = p.Nkv / s - p.kp_first;
     const long long it = item - p.q_items;
-    dst = p.kp + it * kD;
+    const long long bg = it / n_new;
+    const int c = p.kp_first + (int)(it - bg * n_new);
+    dst = p.kp + (bg * p.kp_stride + c) * kD;
     if (!p.paged) {
-      src = p.k + it * s * kD;
+      src = p.k + (bg * p.Nkv + (long long)c * s) * kD;
     } else {
-      const int nkp = p.Nkv / s;
-      const long long bg = it / nkp;
-      const int c = (int)(it - bg * nkp);
       const int b = (int)(bg / p.Hkv), g = (int)(bg - (long long)b * p.Hkv);
       const int tok = c * s, j = tok / p.bk, w = tok - j * p.bk;
       int page = p.page_table[(size_t)b * p.nkb + j];

@@ -1,24 +1,24 @@
-// kap_score: the ranking step of the Kernel-Aware Proxy (CoSA technical
-// summary Sec. 2.2, "Block Ranking" and "HRM Flag Generation").
+// kap_score: the block-scoring step of the Kernel-Aware Proxy (CoSA
+// technical summary Sec. 2.2, "Block Ranking"): pooled scores and MaxPool
+// over the keys of each KV block.
 //
-// One CTA owns 128 pooled query rows of one head.  It streams the pooled
-// keys of the kv-head in tiles of 128 through a TMA ring and contracts them
-// on the tensor cores (tcgen05, bf16 x bf16 -> fp32 in TMEM, two TMEM
-// accumulators so the next tile's MMA overlaps this tile's epilogue):
+// A work item is one run of key tiles (128 pooled keys each) of one row tile
+// (128 pooled query rows) of one head; the key tiles a row tile sees are cut
+// into S items so that short and long rows, and chunks of few queries after
+// a long cache, all spread over the GPU.  Per item, one CTA streams its key
+// tiles through a TMA ring and contracts them on the tensor cores (tcgen05,
+// bf16 x bf16 -> fp32 in TMEM, two TMEM accumulators so the next tile's MMA
+// overlaps this tile's epilogue):
 //   S[r, c]   = Qp[r] . Kp[c]                    (raw pooled scores)
 //   Bs[r, j]  = max over visible c in block j     (MaxPool over keys)
-// Pass 1 stores Bs to workspace and finds each pooled row's max and the
-// first block attaining it (the HRM block).  Pass 2 reads Bs back (each
-// thread its own values, mostly from L2) and emits, per (Q-block, KV block),
-// the aggregated MaxNorm score
-//   score[I, j] = max over the pooled rows r of I of (Bs[r, j] - rowmax[r])
-// and the HRM flag, packed into one ranking key (+1 for HRM blocks, whose
-// score is 0, else the score <= 0) so the sort needs one array.
-// Every selection decision (max, subtract, compare) is taken in fp32.
+// It stores Bs and, per pooled row and column half, the largest Bs of the
+// item and the first block attaining it.  MaxNorm, the HRM flags and the
+// Q-block aggregate need every item of the row and run in kap_sort.
+// Every value is fp32; nothing is rounded after the contraction.
 //
 // Roles: warp 8 issues TMA and MMA; warps 0-7 are the epilogue, two per TMEM
 // lane quarter (row = 32*(warp%4) + lane), each taking one 64-column half of
-// every tile.  The halves' row maxima are merged once, after pass 1.
+// every tile.
 #include <cuda_bf16.h>
 #include "internal.h"
 #include "sm100.cuh"
@@ -40,8 +40,6 @@ struct __align__(8) ScoreSmem {
   uint64_t drained;
   uint32_t tmem_base;
   uint32_t abort;
-  float hmax[2][128];                            // pass-1 row maxima of each column half
-  int harg[2][128];                              // ... and the first block attaining them
 };
 
 // tiles, the control block, and up to 1023 bytes lost aligning the base to 1 KB
@@ -71,13 +69,16 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int heads = p.Hq * p.B;
   const int hb = blockIdx.x % heads;
-  const int R = p.n_row_tiles - 1 - blockIdx.x / heads;       // heaviest row tiles first
+  const int item = blockIdx.x / heads;                         // heaviest row tiles first
+  const int R = p.n_row_tiles - 1 - item / p.splits;
+  const int split = item % p.splits;
   const int h = hb % p.Hq, b = hb / p.Hq, g = h / p.G;
   const int r_first = R * kTileRows;
   const int rows_valid = min(kTileRows, p.nqp - r_first);
-  const int cmax = p.off_p + r_first + rows_valid - 1;        // last pooled key any row here can see
-  const int nT = min(cmax / kTileRows + 1, (p.nkp + kTileRows - 1) / kTileRows);
-  const int U = nT;                                            // MMA tiles (pass 1 only)
+  const int nT = kap_row_tiles_seen(R, p.nqp, p.nkp, p.off_p);
+  int t0, t1;
+  kap_split_range(nT, p.splits, split, t0, t1);
+  const int U = t1 - t0;                                       // key tiles of this item (may be 0)
   constexpr int BPT = kTileRows / KPB;                         // KV blocks per key tile
   constexpr int BPH = BPT / 2;                                 // per 64-column half
 
@@ -106,18 +107,20 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
     tma_prefetch_desc(&tm_qp);
     tma_prefetch_desc(&tm_kp);
     const int qp_y = (b * p.Hq + h) * p.nqp + r_first;
-    const int kp_y0 = (b * p.Hkv + g) * p.nkp;
-    mbar_arrive_expect_tx(&sm->q_full, kTileBytes);
-    tma_load_2d(sQ, &tm_qp, &sm->q_full, 0, qp_y);
-    tma_load_2d(sQ + 16384, &tm_qp, &sm->q_full, 64, qp_y);
+    const int kp_y0 = (b * p.Hkv + g) * p.kp_stride;
+    if (U > 0) {
+      mbar_arrive_expect_tx(&sm->q_full, kTileBytes);
+      tma_load_2d(sQ, &tm_qp, &sm->q_full, 0, qp_y);
+      tma_load_2d(sQ + 16384, &tm_qp, &sm->q_full, 64, qp_y);
+    }
     for (int u = 0; u < 2 && u < U; ++u) {
       uint8_t* dst = sK + u * kTileBytes;
-      const int y = kp_y0 + (u % nT) * kTileRows;
+      const int y = kp_y0 + (t0 + u) * kTileRows;
       mbar_arrive_expect_tx(&sm->k_full[u], kTileBytes);
       tma_load_2d(dst, &tm_kp, &sm->k_full[u], 0, y);
       tma_load_2d(dst + 16384, &tm_kp, &sm->k_full[u], 64, y);
     }
-    bool ok = wait_or_abort(&sm->q_full, 0, abort, p.status, DEV_TIMEOUT_TMA);
+    bool ok = U > 0 && wait_or_abort(&sm->q_full, 0, abort, p.status, DEV_TIMEOUT_TMA);
     const uint32_t idesc = idesc_bf16(128, 128, false, false);
     const uint32_t q_addr = smem_u32(sQ);
     for (int u = 0; ok && u < U; ++u) {
@@ -135,7 +138,7 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
         // refill this stage once the MMA that reads it has completed
         if (!wait_or_abort(&sm->s_full[st], ph, abort, p.status, DEV_TIMEOUT_MMA)) break;
         uint8_t* dst = sK + st * kTileBytes;
-        const int y = kp_y0 + ((u + 2) % nT) * kTileRows;
+        const int y = kp_y0 + (t0 + u + 2) * kTileRows;
         mbar_arrive_expect_tx(&sm->k_full[st], kTileBytes);
         tma_load_2d(dst, &tm_kp, &sm->k_full[st], 0, y);
         tma_load_2d(dst + 16384, &tm_kp, &sm->k_full[st], 64, y);
@@ -151,19 +154,13 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
     const int r = r_first + row;
     const bool row_ok = row < rows_valid;
     const int climit = p.off_p + r;
-    const int I = r / p.rpq;
-    const int last_tok = min((I + 1) * p.bq, p.Nq) - 1;
-    const int n_I = min(p.nkb, (p.Nkv - p.Nq + last_tok) / p.bk + 1);
-    const bool qblock_ok = I < p.nqb;
-    const size_t rank_row = ((size_t)(b * p.Hq + h) * p.nqb + I) * p.nkb;
-    const int gl = lane % p.rpq;                // position inside the Q-block's lane group
     float rowmax = -INFINITY;
     int argj = -1;
     // this row's Bs, [nKB][128 rows] per (head, row tile): coalesced across the warp
-    float* bs_row = p.bs + ((size_t)(b * p.Hq + h) * p.n_row_tiles + R) * p.nkb * kTileRows + row;
+    float* bs_row = p.bs + ((size_t)hb * p.n_row_tiles + R) * p.nkb * kTileRows + row;
     for (int u = 0; u < U; ++u) {
       const int st = u & 1;
-      const int T = u % nT;
+      const int T = t0 + u;
       const bool got = wait_or_abort(&sm->s_full[st], (u >> 1) & 1, abort, p.status, DEV_TIMEOUT_MMA);
       tc_fence_after();
       float bsv[BPH];
@@ -197,40 +194,11 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
 #pragma unroll
       for (int jh = 0; jh < BPH; ++jh)
         if (bsv[jh] > rowmax) { rowmax = bsv[jh]; argj = j0 + jh; }
-      if (u == nT - 1) {
-        // merge the two halves: the larger max; on a tie the smaller block index
-        sm->hmax[half][row] = rowmax;
-        sm->harg[half][row] = argj;
-        named_barrier(1, 32 * kEpiWarps);
-        const float m0 = sm->hmax[0][row], m1 = sm->hmax[1][row];
-        const int a0 = sm->harg[0][row], a1 = sm->harg[1][row];
-        rowmax = fmaxf(m0, m1);
-        argj = (m0 > m1) ? a0 : (m1 > m0) ? a1 : min(a0, a1);
-      }
     }
-    // pass 2: MaxNorm, HRM flags and the Q-block aggregate from the stored Bs
-    // (values this thread wrote itself)
-    for (int T = 0; T < nT; ++T) {
-      const int j0 = T * BPT + half * BPH;
-      float bsv[BPH];
-#pragma unroll
-      for (int jh = 0; jh < BPH; ++jh) bsv[jh] = j0 + jh < p.nkb ? bs_row[(size_t)(j0 + jh) * kTileRows] : -INFINITY;
-      // HRM: the Q-block's flags for this half-tile, as a bit mask OR-ed over its rows
-      uint32_t bits = (argj >= j0 && argj < j0 + BPH) ? 1u << (argj - j0) : 0u;
-      for (int o = 1; o < p.rpq; o <<= 1) bits |= __shfl_xor_sync(0xffffffffu, bits, o);
-#pragma unroll
-      for (int jh = 0; jh < BPH; ++jh) {
-        const int j = j0 + jh;
-        float z = (row_ok && bsv[jh] != -INFINITY) ? __fsub_rn(bsv[jh], rowmax) : -INFINITY;
-        for (int o = 1; o < p.rpq; o <<= 1) z = fmaxf(z, __shfl_xor_sync(0xffffffffu, z, o));
-        const uint32_t flag = (bits >> jh) & 1u;
-        if (qblock_ok && (jh % p.rpq) == gl && j < n_I) {
-          p.rank[rank_row + j] = flag ? 1.0f : z;
-          if (p.block_score) p.block_score[rank_row + j] = z;
-          if (p.hrm_flags) p.hrm_flags[rank_row + j] = (uint8_t)flag;
-        }
-      }
-    }
+    // this item's row maximum for this column half (-inf / -1 when it saw nothing)
+    const size_t pi = ((((size_t)hb * p.n_row_tiles + R) * p.splits + split) * 2 + half) * kTileRows + row;
+    p.part_max[pi] = rowmax;
+    p.part_arg[pi] = argj;
   }
   tc_fence_before();
   __syncthreads();
@@ -244,7 +212,7 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
 
 cudaError_t launch_kap_score(const CUtensorMap& tm_qp, const CUtensorMap& tm_kp, const ScoreParams& p,
                              cudaStream_t st) {
-  const unsigned grid = (unsigned)(p.n_row_tiles * p.Hq * p.B);
+  const unsigned grid = (unsigned)(p.n_row_tiles * p.splits * p.Hq * p.B);
   if (grid == 0) return cudaSuccess;
 #define COSA_LAUNCH_SCORE(K)                                                                          \
   case K: {                                                                                           \

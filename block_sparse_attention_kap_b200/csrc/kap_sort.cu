@@ -1,17 +1,24 @@
-// kap_sort: flag-grouped sorting of the Kernel-Aware Proxy (CoSA technical
-// summary Sec. 2.2): per (head, Q-block), the causally visible KV blocks are
-// ordered HRM blocks first, then by estimated score, ties by block index,
-// and the first k_I = max(1, ceil(n_I * budget)) form the computation-order
-// mask M_KAP.
+// kap_sort: the ranking and flag-grouped sorting of the Kernel-Aware Proxy
+// (CoSA technical summary Sec. 2.2, "Block Ranking", "HRM Flag Generation"
+// and the sort): per (head, Q-block), from the max-pooled block scores Bs of
+// its pooled rows (kap_score),
+//   rowmax[r]  = max_j Bs[r, j]; HRM block of r = first j attaining it
+//   score[j]   = max over the Q-block's rows r of (Bs[r, j] - rowmax[r])
+// (MaxNorm, then the aggregate), and the causally visible blocks are ordered
+// HRM blocks first, then by score, ties by block index; the first
+// k_I = max(1, ceil(n_I * budget)) form the computation-order mask M_KAP.
+// Every value is fp32 and every decision is taken on fp32 values.
 //
 // One warp per (b, h, Q-block), several per CTA, synchronised only with
-// __syncwarp.  Each block's ranking key (+1 for HRM blocks, else its score
-// <= 0, written by kap_score) is mapped to an order-preserving 32-bit
-// integer.  A 4-pass, 8-bit radix select (per-warp shared-memory histogram)
-// finds the k-th largest value T; the blocks above T plus the lowest-indexed
-// blocks equal to T are compacted in index order with warp ballots, and only
-// those k keys -- packed with the inverted block index so ties resolve to
-// the smaller index -- are sorted by a bitonic network in shared memory.
+// __syncwarp.  The row maxima come from kap_score's per-item partial maxima
+// (ties resolved to the smaller block index).  Each block's ranking key (+1
+// for HRM blocks, else its score <= 0) is mapped to an order-preserving
+// 32-bit integer.  A 4-pass, 8-bit radix select (per-warp shared-memory
+// histogram) finds the k-th largest value T; the blocks above T plus the
+// lowest-indexed blocks equal to T are compacted in index order with warp
+// ballots, and only those k keys -- packed with the inverted block index so
+// ties resolve to the smaller index -- are sorted by a bitonic network in
+// shared memory.
 #include "internal.h"
 
 namespace cosa {
@@ -37,6 +44,7 @@ __host__ __device__ __forceinline__ size_t warp_smem(int nkb, int pk) {
   return 1024 + align16((size_t)nkb * 4) + (size_t)pk * 8;
 }
 
+template <int RPQ>
 __global__ void __launch_bounds__(32 * kMaxWarps) kap_sort_kernel(SortParams p, int pk, int rows) {
   extern __shared__ __align__(16) uint8_t dyn[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -50,17 +58,62 @@ __global__ void __launch_bounds__(32 * kMaxWarps) kap_sort_kernel(SortParams p, 
   const unsigned lt_mask = (1u << lane) - 1u;
 
   const int I = row % p.nqb;
+  const int hb = row / p.nqb;                    // b * Hq + h
   const int n = causal_blocks(I, p.Nq, p.Nkv, p.bq, p.bk, p.nkb);
   int k = (int)(((long long)n * p.bp + 9999) / 10000);
   k = max(1, min(k, n));
-  const float* rk = p.rank + (size_t)row * p.nkb;
-  const uint32_t hrm_key = orderable(1.0f);
 
+  // ------------------------------------------------------------ row maxima of the Q-block's pooled rows
+  const int r_abs0 = I * RPQ;                    // first pooled row (a Q-block never straddles row tiles)
+  const int R = r_abs0 / kTileRows, row0 = r_abs0 % kTileRows;
+  float my_max = -INFINITY;
+  int my_arg = -1;
+  if (lane < RPQ) {
+    const size_t base = ((size_t)hb * p.n_row_tiles + R) * p.splits * 2 * kTileRows + row0 + lane;
+    for (int q = 0; q < 2 * p.splits; ++q) {
+      const float m = p.part_max[base + (size_t)q * kTileRows];
+      const int a = p.part_arg[base + (size_t)q * kTileRows];
+      if (m > my_max || (m == my_max && a >= 0 && (my_arg < 0 || a < my_arg))) { my_max = m; my_arg = a; }
+    }
+  }
+  float rmax[RPQ];
+  int rarg[RPQ];
+#pragma unroll
+  for (int i = 0; i < RPQ; ++i) {
+    rmax[i] = __shfl_sync(full, my_max, i);
+    rarg[i] = __shfl_sync(full, my_arg, i);
+  }
+
+  // ------------------------------------------------------------ MaxNorm, aggregate, HRM -> ranking keys
+  const float* bs = p.bs + ((size_t)hb * p.n_row_tiles + R) * p.nkb * kTileRows + row0;
+  const size_t out_row = (size_t)row * p.nkb;
+  const uint32_t hrm_key = orderable(1.0f);
   int hrm = 0;
-  for (int i = lane; i < n; i += 32) {
-    const uint32_t h = orderable(rk[i]);
-    hi[i] = h;
-    hrm += (h == hrm_key);
+  for (int j = lane; j < n; j += 32) {
+    float v[RPQ];
+    const float* src = bs + (size_t)j * kTileRows;
+    if constexpr (RPQ % 4 == 0) {
+#pragma unroll
+      for (int i = 0; i < RPQ; i += 4) {
+        const float4 f = __ldg(reinterpret_cast<const float4*>(src + i));
+        v[i] = f.x; v[i + 1] = f.y; v[i + 2] = f.z; v[i + 3] = f.w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < RPQ; ++i) v[i] = __ldg(src + i);
+    }
+    float z = -INFINITY;
+    bool flag = false;
+#pragma unroll
+    for (int i = 0; i < RPQ; ++i) {
+      if (v[i] != -INFINITY) z = fmaxf(z, __fsub_rn(v[i], rmax[i]));
+      flag |= rarg[i] == j;
+    }
+    const uint32_t h = flag ? hrm_key : orderable(z);
+    hi[j] = h;
+    hrm += flag;
+    if (p.block_score) p.block_score[out_row + j] = z;
+    if (p.hrm_flags) p.hrm_flags[out_row + j] = (uint8_t)flag;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) hrm += __shfl_xor_sync(full, hrm, o);
@@ -190,10 +243,25 @@ cudaError_t launch_kap_sort(const SortParams& p, cudaStream_t st) {
   warps = warps < 1 ? 1 : (warps > kMaxWarps ? kMaxWarps : warps);
   const size_t smem = per_warp * warps;
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(kap_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)((rows + warps - 1) / warps);
-  kap_sort_kernel<<<grid, 32 * warps, smem, st>>>(p, pk, rows);
+#define COSA_LAUNCH_SORT(R)                                                                           \
+  case R: {                                                                                           \
+    cudaError_t e = cudaFuncSetAttribute(kap_sort_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                                         (int)smem);                                                  \
+    if (e != cudaSuccess) return e;                                                                   \
+    kap_sort_kernel<R><<<grid, 32 * warps, smem, st>>>(p, pk, rows);                                  \
+    break;                                                                                            \
+  }
+  switch (p.rpq) {
+    COSA_LAUNCH_SORT(2)
+    COSA_LAUNCH_SORT(4)
+    COSA_LAUNCH_SORT(8)
+    COSA_LAUNCH_SORT(16)
+    COSA_LAUNCH_SORT(32)
+    default:
+      return cudaErrorInvalidValue;
+  }
+#undef COSA_LAUNCH_SORT
   return cudaGetLastError();
 }
 

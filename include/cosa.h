@@ -78,8 +78,8 @@ COSA_API int cosa_num_kblocks(const cosa_shape* shape);
 COSA_API int cosa_kmax(const cosa_shape* shape, double budget);
 
 /* Bytes of device workspace cosa_plan needs (pooled Q, pooled K, the
- * per-(head, Q-block) block ranking and the max-pooled block scores of every
- * pooled query row).  0 for an invalid shape. */
+ * max-pooled block scores of every pooled query row and partial row maxima).
+ * 0 for an invalid shape. */
 COSA_API size_t cosa_plan_workspace_bytes(const cosa_shape* shape);
 
 /* KAP, stage 1 (Sec. 2.2): downsample Q and K (mean of `stride` consecutive
@@ -102,6 +102,62 @@ COSA_API cosa_status cosa_plan(const cosa_shape* shape, const void* q, const voi
                       double budget, int kmax, int32_t* order, int32_t* count, int32_t* hrm_count,
                       float* block_score, uint8_t* hrm_flags, void* workspace, size_t ws_bytes,
                       uint32_t* dev_status, cudaStream_t stream);
+
+/* cosa_plan for one chunk of a chunked prefill, with the pooled keys kept
+ * from one chunk to the next.  In chunked prefill ("CompactAttention:
+ * Accelerating Chunked Prefill with Block-Union KV Selection", selection
+ * stage and evaluation setup) each chunk of Nq new queries attends to a
+ * cache of Nkv keys that holds every earlier chunk plus its own; re-pooling
+ * the whole cache per chunk reads all of K again.  Here the pooled keys live
+ * in a caller-owned cache and only the keys not yet pooled are read.
+ *  kp_cache    [B, Hkv, kp_capacity, d] bf16, device, 16-byte aligned,
+ *              owned by the caller and kept across chunks.  Row c of a head
+ *              holds the mean of keys stride*c .. stride*c + stride - 1.
+ *  kp_capacity pooled-key rows per head in the cache (>= Nkv / stride).
+ *  kp_valid    rows 0 .. kp_valid-1 of every head were written by an
+ *              earlier call for the same keys and are used as they are;
+ *              rows kp_valid .. Nkv/stride - 1 are pooled from k (contiguous
+ *              or paged, as for cosa_plan) and written to the cache before
+ *              scoring.  0 <= kp_valid <= Nkv / stride; kp_valid = 0 pools
+ *              every key.  Chunk after chunk, pass the previous call's
+ *              Nkv / stride.
+ * Every other argument and result is cosa_plan's, and the results are
+ * bit-identical to cosa_plan's on the same q and k (pooling is
+ * deterministic per row).  The workspace is sized by
+ * cosa_plan_workspace_bytes (its pooled-key region goes unused).  Returns
+ * COSA_EINVAL for a null cache or kp_capacity / kp_valid out of range,
+ * COSA_EALIGN for a misaligned cache. */
+COSA_API cosa_status cosa_plan_chunk(const cosa_shape* shape, const void* q, const void* k,
+                                     const int32_t* page_table, void* kp_cache, int kp_capacity, int kp_valid,
+                                     double budget, int kmax, int32_t* order, int32_t* count,
+                                     int32_t* hrm_count, float* block_score, uint8_t* hrm_flags,
+                                     void* workspace, size_t ws_bytes, uint32_t* dev_status,
+                                     cudaStream_t stream);
+
+/* Block union ("CompactAttention: Accelerating Chunked Prefill with
+ * Block-Union KV Selection", method, selection stage): turn a per-head
+ * selection into one KV block table per (batch, kv-head group), the union
+ * over every Q-block of the call (the chunk) and every query head sharing
+ * the kv-head.  Every block any of them selected is in the table, no other
+ * block is, and the table ascends.
+ *  order, count  [B, Hq, nQB, kmax], [B, Hq, nQB] int32 in: the selection
+ *                (typically cosa_plan's M_KAP); entries at or beyond count
+ *                and indices outside [0, nKB) are ignored; count is clamped
+ *                to [0, kmax].
+ *  table         [B, Hkv, nKB] int32 out: the union, ascending, padded -1.
+ *  table_len     [B, Hkv] int32 out: its length.
+ *  union_order   [B, Hq, nQB, union_kmax] int32 out (nullable, together with
+ *                union_count): per Q-block, the table entries it can see
+ *                causally, ascending, padded -1 -- an order cosa_attend
+ *                executes (skip_eps = 0 gives the dense attention over the
+ *                union the paper runs).  union_kmax must be >= the number of
+ *                causally visible blocks of the last Q-block.
+ *  union_count   [B, Hq, nQB] int32 out: length of each union_order row.
+ * Returns COSA_EINVAL for null outputs, a missing order/count, or a
+ * union_kmax that is too small. */
+COSA_API cosa_status cosa_block_union(const cosa_shape* shape, const int32_t* order, const int32_t* count,
+                                      int kmax, int32_t* table, int32_t* table_len, int32_t* union_order,
+                                      int32_t* union_count, int union_kmax, cudaStream_t stream);
 
 /* Fill `order`/`count` with every causally visible block of each Q-block in
  * natural order (0, 1, ..., n_I - 1): the dense path, which cosa_attend runs

@@ -60,6 +60,40 @@ def round_bf16(x: torch.Tensor) -> torch.Tensor:
     return torch.where(torch.isfinite(x), r, x)
 
 
+def block_union(wl, order: torch.Tensor, count: torch.Tensor):
+    """Block union of CompactAttention's selection stage ("CompactAttention:
+    Accelerating Chunked Prefill with Block-Union KV Selection", method): the
+    KV block table of (batch b, kv-head g) is the set of blocks that any
+    Q-block of any query head h with h // G == g selected, in ascending
+    order.  order [B*Hq*nQB, kmax] and count [B*Hq*nQB] in (b, h, I)
+    row-major order.  Returns (tables: list over (b, g) of sorted lists,
+    per-row visible prefixes: list over (b, h, I) rows)."""
+    B, Hq, Hkv, nqb, nkb = wl.B, wl.Hq, wl.Hkv, wl.n_qblocks, wl.n_kblocks
+    G = Hq // Hkv
+    order = order.view(B, Hq, nqb, -1)
+    count = count.view(B, Hq, nqb)
+    kmax_ = order.shape[-1]
+    tables = []
+    for b in range(B):
+        for g in range(Hkv):
+            chosen = set()
+            for h in range(g * G, (g + 1) * G):
+                for I in range(nqb):
+                    c = min(max(int(count[b, h, I]), 0), kmax_)
+                    for j in order[b, h, I, :c].tolist():
+                        if 0 <= j < nkb:
+                            chosen.add(j)
+            tables.append(sorted(chosen))
+    rows = []
+    for b in range(B):
+        for h in range(Hq):
+            tab = tables[b * Hkv + h // G]
+            for I in range(nqb):
+                lim = lib().oracle_causal_blocks(ctypes.byref(shape_of(wl)), I)   # blocks 0..lim-1 visible
+                rows.append([j for j in tab if j < lim])
+    return tables, rows
+
+
 def shape_of(wl) -> OrShape:
     return OrShape(wl.B, wl.Hq, wl.Hkv, wl.Nq, wl.Nkv, wl.d, wl.bq, wl.bk, wl.stride,
                    1 if wl.paged else 0, wl.num_pages)

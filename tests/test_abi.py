@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(cosa):
 
 
 def test_version(cosa):
-    assert cosa.cosa_version() == 100
+    assert cosa.cosa_version() == 101
 
 
 @pytest.mark.parametrize("name", list(synth.WORKLOADS))
@@ -93,6 +93,45 @@ def test_plan_argument_errors_return_before_launch(cosa):
     assert _raw_plan(cosa, paged, kmax=km) == 1                 # paged without a page table
     empty = cosa.make_shape(1, 4, 2, 0, 512, 128, 128, 64, 16)
     assert _raw_plan(cosa, empty, q=None, k=None, order=None, count=None, ws=None, kmax=0) == 0
+
+
+def test_plan_chunk_argument_errors_return_before_launch(cosa):
+    lib = cosa._lib
+    s = cosa.make_shape(1, 4, 2, 256, 1024, 128, 128, 64, 16)     # 64 pooled keys per head
+    km = cosa.cosa_kmax(s, 0.1)
+    P = 1 << 20
+    ws_bytes = cosa.cosa_plan_workspace_bytes(s)
+
+    def call(cache=P, cap=64, valid=48, q=P, kmax=km, ws_bytes=ws_bytes, shape=s):
+        return lib.cosa_plan_chunk(ctypes.byref(shape), q, P, None, cache, cap, valid, 0.1, kmax, P, P, None,
+                                   None, None, P, ws_bytes, None, None)
+    assert call(cache=None) == 1                  # EINVAL: no cache
+    assert call(cap=63) == 1                      # capacity below Nkv / stride
+    assert call(valid=-1) == 1
+    assert call(valid=65) == 1                    # more valid rows than keys
+    assert call(cache=P + 8) == 2                 # EALIGN
+    assert call(q=None) == 1
+    assert call(kmax=km - 1) == 1
+    assert call(ws_bytes=256) == 4                # EWORKSPACE
+    assert call(shape=cosa.make_shape(1, 4, 2, 256, 1000, 128, 128, 64, 16)) == 3
+    assert call(shape=cosa.make_shape(1, 4, 2, 0, 1024, 128, 128, 64, 16), q=None, cache=None) == 0
+
+
+def test_block_union_argument_errors_return_before_launch(cosa):
+    lib = cosa._lib
+    s = cosa.make_shape(1, 4, 2, 256, 768, 128, 128, 128, 16)      # nKB = 6; the last Q-block sees 6
+    P = 1 << 20
+
+    def call(order=P, count=P, kmax=4, table=P, tlen=P, uo=P, uc=P, ukmax=6, shape=s):
+        return lib.cosa_block_union(ctypes.byref(shape), order, count, kmax, table, tlen, uo, uc, ukmax, None)
+    assert call(table=None) == 1
+    assert call(tlen=None) == 1
+    assert call(order=None) == 1
+    assert call(kmax=-1) == 1
+    assert call(ukmax=5) == 1                     # too short for the last Q-block's visible blocks
+    assert call(uc=None) == 1                     # union_order without union_count
+    assert call(shape=cosa.make_shape(1, 4, 3, 256, 768, 128, 128, 128, 16)) == 3
+    assert call(shape=cosa.make_shape(0, 4, 2, 256, 768, 128, 128, 128, 16), table=None) == 0
 
 
 def test_attend_argument_errors_return_before_launch(cosa):

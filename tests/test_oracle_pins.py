@@ -468,3 +468,56 @@ def test_mass_recall_identity():
             assert torch.allclose(recall[i], mass, atol=1e-12, rtol=1e-9)
             i += 1
     assert bool((recall <= 1 + 1e-12).all()) and bool((recall > 0).all())
+
+
+# ----------------------------------------------------------------- block union (CompactAttention)
+
+def test_block_union_hand_example():
+    """CompactAttention, method, selection stage: per (batch, kv-head) the
+    union over the chunk's Q-blocks and the group's heads.  Worked by hand:
+    Hq=4, Hkv=2 (heads 0,1 -> group 0; 2,3 -> group 1), two Q-blocks of 128
+    after 512 cached keys, blocks of 128 (nKB = 6; Q-block 0 sees blocks
+    0..4, Q-block 1 sees 0..5).  Entries past count, negative entries and
+    indices >= nKB are not selections; count is clamped to kmax."""
+    wl = tiny(Hq=4, Hkv=2, Nq=256, Nkv=768, bq=128, bk=128)
+    order = torch.tensor([[3, 1, -1], [0, 5, 2],      # h0: I0 {3,1}, I1 {0,5,2}
+                          [4, 9, 9], [1, 7, 2],       # h1: I0 {4} (9 past count), I1 {1} (7 out of range)
+                          [6, -1, -1], [2, 3, 12],    # h2: I0 {} (6 out of range), I1 {2,3}
+                          [0, 0, 0], [8, 0, 0]],      # h3: I0 count 0, I1 count 5 -> 3: {0}
+                         dtype=torch.int32)
+    count = torch.tensor([2, 3, 1, 2, 1, 3, 0, 5], dtype=torch.int32)
+    tables, rows = oracle.block_union(wl, order, count)
+    assert tables == [[0, 1, 2, 3, 4, 5], [0, 2, 3]]
+    assert rows == [[0, 1, 2, 3, 4], [0, 1, 2, 3, 4, 5]] * 2 + [[0, 2, 3], [0, 2, 3]] * 2
+
+
+def test_block_union_properties_random():
+    """Coverage (every selected block of the group is in its table),
+    minimality (every table entry was selected by some Q-block or head of the
+    group), ascending order, and each row's prefix = the table entries the
+    Q-block can see -- checked against a boolean selection matrix built
+    independently of the oracle's sets."""
+    rng = torch.Generator().manual_seed(11)
+    wl = tiny(B=2, Hq=8, Hkv=2, Nq=384, Nkv=2048, bq=128, bk=64)
+    n, nkb, km = wl.B * wl.Hq * wl.n_qblocks, wl.n_kblocks, 9
+    order = torch.randint(-3, nkb + 3, (n, km), generator=rng, dtype=torch.int32)
+    count = torch.randint(-1, km + 3, (n,), generator=rng, dtype=torch.int32)
+    tables, rows = oracle.block_union(wl, order, count)
+    G = wl.Hq // wl.Hkv
+    sel = torch.zeros(wl.B, wl.Hkv, nkb, dtype=torch.bool)
+    o4 = order.view(wl.B, wl.Hq, wl.n_qblocks, km)
+    c3 = count.view(wl.B, wl.Hq, wl.n_qblocks).clamp(0, km)
+    t = torch.arange(km)
+    valid = (t < c3[..., None]) & (o4 >= 0) & (o4 < nkb)
+    for b in range(wl.B):
+        for h in range(wl.Hq):
+            sel[b, h // G, o4[b, h][valid[b, h]].long()] = True
+    off = wl.Nkv - wl.Nq
+    for b in range(wl.B):
+        for g in range(wl.Hkv):
+            tab = tables[b * wl.Hkv + g]
+            assert tab == torch.nonzero(sel[b, g]).view(-1).tolist()
+            for h in range(g * G, (g + 1) * G):
+                for I in range(wl.n_qblocks):
+                    last_key = off + min((I + 1) * wl.bq, wl.Nq) - 1
+                    assert rows[(b * wl.Hq + h) * wl.n_qblocks + I] == [j for j in tab if j * wl.bk <= last_key]
