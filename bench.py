@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--budget B] [--eps E] [--impl cosa|reference]
-                    [--sweep | --chunked]
+                    [--sweep | --chunked | --decode]
 
 One step = one pass of the whole hot path over one batch of synthetic
 input: cosa_plan (kap_pool, kap_score, kap_sort) then cosa_attend
@@ -59,6 +59,9 @@ def parse():
     ap.add_argument("--chunked", action="store_true",
                     help="chunked prefill: KAP with the pooled keys kept across chunks (cosa_plan_chunk) "
                          "against KAP that re-pools the whole cache (cosa_plan), one line (no headline line)")
+    ap.add_argument("--decode", action="store_true",
+                    help="one decode step per head after the workload's cache: cosa_decode_plan + cosa_attend "
+                         "(Nq = 1) against the dense decode step, one line (no headline line)")
     ap.add_argument("--sweep", action="store_true",
                     help="one line per budget of the workload: latency, in-kernel skip fraction and error "
                          "against the dense path (no headline line)")
@@ -370,6 +373,73 @@ def run_chunked(args, wl, budget, eps):
         "effective_tflops_chunk": wl.dense_causal_flops() / ((chunk_ms + attend_ms) * 1e-3) / 1e12}), flush=True)
 
 
+# ----------------------------------------------------------------- decode step
+
+def run_decode(args, wl, budget, eps):
+    """One decode step: the last query row of every head of the workload is
+    the new token (position Nkv-1); the pooled keys are already cached, as
+    after a prefill with cosa_plan_chunk.  Times the proxy (cosa_decode_plan)
+    and the attention (cosa_attend with Nq = 1), against the dense decode
+    step (every block, eps 0) on the same kernel; reports the K/V bytes the
+    sparse step reads and its error against the dense step."""
+    import block_sparse_attention_kap_b200 as cosa
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    inp = synth.generate(wl)
+    q = inp.q[:, :, -1:, :].contiguous().to(dev)                 # [B, Hq, 1, d]
+    k, v = inp.k.to(dev), inp.v.to(dev)
+    pt = inp.page_table.to(dev) if inp.page_table is not None else None
+    shape = cosa.make_shape(wl.B, wl.Hq, wl.Hkv, 1, wl.Nkv, wl.d, 128, wl.bk, wl.stride, wl.paged,
+                            wl.num_pages if wl.paged else 0)
+    m = cosa.CoSA(shape, device=dev)
+    nkp = wl.Nkv // wl.stride
+    cache = torch.empty(wl.B, wl.Hkv, nkp, wl.d, dtype=torch.bfloat16, device=dev)
+    plan = m.decode_plan(q, k, budget, cache, 0, page_table=pt)   # fills the pooled-key cache
+    order, count = plan["order"], plan["count"]
+    km = order.shape[-1]
+    out = torch.empty(wl.B, wl.Hq, 1, wl.d, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / args.steps
+
+    plan_ms = timed(lambda: cosa.cosa_decode_plan(shape, q, k, pt, cache, nkp, budget, km, order, count,
+                                                  plan["hrm_count"], None, None, stream))
+    attend_ms = timed(lambda: cosa.cosa_attend(shape, q, k, v, pt, order, count, km, eps, out, None, None,
+                                               m.status, stream))
+    d_order, d_count = m.dense_order()
+    dense_ms = timed(lambda: cosa.cosa_attend(shape, q, k, v, pt, d_order, d_count, d_order.shape[-1], 0.0, out,
+                                              None, None, m.status, stream))
+    res = m.attend(q, k, v, order, count, eps, page_table=pt, skip_bits=True)
+    dense_out = m.attend(q, k, v, d_order, d_count, 0.0, page_table=pt)["out"].float()
+    torch.cuda.synchronize()
+    assert m.device_status() == 0
+    sel = int(count.sum().item())
+    skipped = int(cosa.unpack_skip_bits(res["skip_bits"], km).sum().item())
+    tile = wl.bk * wl.d * 2
+    sparse_bytes = tile * (sel + (sel - skipped))                  # K of every visit, V of computed ones
+    dense_bytes = 2 * tile * int(d_count.sum().item())
+    err = (res["out"].float() - dense_out).abs()
+    rows = wl.B * wl.Hq
+    print(json.dumps({
+        "kind": "decode", "workload": wl.name, "rows": rows, "Nkv": wl.Nkv, "budget": budget, "eps": eps,
+        "plan_ms": plan_ms, "attend_ms": attend_ms, "step_ms": plan_ms + attend_ms, "dense_step_ms": dense_ms,
+        "speedup_vs_dense": dense_ms / (plan_ms + attend_ms),
+        "selected_blocks": sel, "skipped_in_kernel_frac": skipped / max(1, sel),
+        "kv_bytes": {"sparse": sparse_bytes, "dense": dense_bytes},
+        "attend_gbs_requested": sparse_bytes / (attend_ms * 1e-3) / 1e9,
+        "err_vs_dense": {"max_abs": err.max().item(), "mean_abs": err.mean().item()}}), flush=True)
+
+
 # ----------------------------------------------------------------- GPU arm
 
 def main():
@@ -388,6 +458,9 @@ def main():
         return
     if args.chunked:
         run_chunked(args, wl, budget, eps)
+        return
+    if args.decode:
+        run_decode(args, wl, budget, eps)
         return
     if args.warmup < 3:
         args.warmup = 3

@@ -58,6 +58,8 @@ _lib.cosa_plan_chunk.argtypes = [_S, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int,
                                  _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]
 _lib.cosa_dense_order.argtypes = [_S, ctypes.c_int, _P, _P, _P]
 _lib.cosa_block_union.argtypes = [_S, _P, _P, ctypes.c_int, _P, _P, _P, _P, ctypes.c_int, _P]
+_lib.cosa_decode_plan.argtypes = [_S, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
+                                  _P, _P, _P, _P, _P, _P]
 _lib.cosa_plan_static.argtypes = [_S, _P, _P, _P, ctypes.c_double, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P]
 _lib.cosa_attend.argtypes = [_S, _P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_double, _P, _P, _P, _P, _P]
 _lib.cosa_skip_threshold.argtypes = [ctypes.c_double, ctypes.c_int]
@@ -67,7 +69,7 @@ _lib.cosa_status_string.restype = ctypes.c_char_p
 
 EXPORTS = ("cosa_num_qblocks", "cosa_num_kblocks", "cosa_kmax", "cosa_plan_workspace_bytes", "cosa_plan",
            "cosa_dense_order", "cosa_attend", "cosa_skip_threshold", "cosa_status_string", "cosa_version",
-           "cosa_plan_static", "cosa_plan_chunk", "cosa_block_union")
+           "cosa_plan_static", "cosa_plan_chunk", "cosa_block_union", "cosa_decode_plan")
 STATIC_SCRATCH_BYTES = 64 << 20
 
 
@@ -179,6 +181,23 @@ def cosa_dense_order(shape: cosa_shape, kmax: int, order, count, stream=None) ->
                                  _ptr(count, "count", torch.int32), _stream(stream)), "cosa_dense_order")
 
 
+def cosa_decode_plan(shape: cosa_shape, q, k, page_table, kp_cache, kp_valid: int, budget: float, kmax: int,
+                     order, count, hrm_count=None, block_score=None, hrm_flags=None, stream=None) -> None:
+    """The proxy for one decode step (shape.Nq == 1): q [B, Hq, 1, d]; the
+    pooled keys come from kp_cache [B, Hkv, capacity, d] (rows below
+    kp_valid reused, the rest pooled from k first)."""
+    if kp_cache is not None and kp_cache.dim() != 4:
+        raise ValueError("kp_cache must be [B, Hkv, capacity, d]")
+    cap = kp_cache.shape[2] if kp_cache is not None else 0
+    _check(_lib.cosa_decode_plan(ctypes.byref(shape), _ptr(q, "q", torch.bfloat16), _ptr(k, "k", torch.bfloat16),
+                                 _ptr(page_table, "page_table", torch.int32),
+                                 _ptr(kp_cache, "kp_cache", torch.bfloat16), cap, kp_valid, budget, kmax,
+                                 _ptr(order, "order", torch.int32), _ptr(count, "count", torch.int32),
+                                 _ptr(hrm_count, "hrm_count", torch.int32),
+                                 _ptr(block_score, "block_score", torch.float32),
+                                 _ptr(hrm_flags, "hrm_flags", torch.uint8), _stream(stream)), "cosa_decode_plan")
+
+
 def cosa_block_union(shape: cosa_shape, order, count, kmax: int, table, table_len, union_order=None,
                      union_count=None, stream=None) -> None:
     union_kmax = union_order.shape[-1] if union_order is not None else 0
@@ -267,6 +286,24 @@ class CoSA:
             res.update(block_score=bs, hrm=hf)
         return res
 
+    def decode_plan(self, q, k, budget: float, kp_cache, kp_valid: int, page_table=None, scores: bool = False,
+                    stream=None):
+        """The proxy for one decode step (shape.Nq == 1)."""
+        s = self.shape
+        km = max(cosa_kmax_decode(s, budget), 1)
+        order = torch.empty(s.B, s.Hq, 1, km, dtype=torch.int32, device=self.device)
+        count = torch.empty(s.B, s.Hq, 1, dtype=torch.int32, device=self.device)
+        hrm = torch.empty(s.B, s.Hq, 1, dtype=torch.int32, device=self.device)
+        bs = hf = None
+        if scores:
+            bs = torch.empty(s.B, s.Hq, 1, self.nkb, dtype=torch.float32, device=self.device)
+            hf = torch.empty(s.B, s.Hq, 1, self.nkb, dtype=torch.uint8, device=self.device)
+        cosa_decode_plan(s, q, k, page_table, kp_cache, kp_valid, budget, km, order, count, hrm, bs, hf, stream)
+        res = dict(order=order, count=count, hrm_count=hrm)
+        if scores:
+            res.update(block_score=bs, hrm=hf)
+        return res
+
     def block_union(self, order, count, expand: bool = True, stream=None):
         """Per-(batch, kv-head) union of a selection over the Q-blocks and the
         heads of each group; with expand, also the causally visible prefix
@@ -306,6 +343,13 @@ class CoSA:
 
     def device_status(self) -> int:
         return int(self.status.item())
+
+
+def cosa_kmax_decode(shape: cosa_shape, budget: float) -> int:
+    """Blocks a decode step keeps: max(1, ceil(nKB * round(budget * 1e4) / 1e4))."""
+    nkb = cosa_num_kblocks(shape)
+    bp = int(round(budget * 10000))
+    return max(1, min(nkb, -(-nkb * bp // 10000)))
 
 
 def shape_of_workload(wl) -> cosa_shape:

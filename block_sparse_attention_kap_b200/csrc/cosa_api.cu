@@ -10,6 +10,7 @@
 #include "cosa.h"
 #include "internal.h"
 #include "block_union.h"
+#include "decode.h"
 
 using namespace cosa;
 
@@ -284,6 +285,50 @@ cosa_status cosa_dense_order(const cosa_shape* shape, int kmax, int32_t* order, 
   if (kmax < causal_blocks(shape, n_qblocks(shape) - 1)) return COSA_EINVAL;
   return launch_status(launch_dense_order(rows, n_qblocks(shape), n_kblocks(shape), shape->Nq, shape->Nkv,
                                           shape->bq, shape->bk, kmax, order, count, stream));
+}
+
+cosa_status cosa_decode_plan(const cosa_shape* shape, const void* q, const void* k, const int32_t* page_table,
+                             void* kp_cache, int kp_capacity, int kp_valid, double budget, int kmax,
+                             int32_t* order, int32_t* count, int32_t* hrm_count, float* block_score,
+                             uint8_t* hrm_flags, cudaStream_t stream) {
+  cosa_status st = check_shape(shape);
+  if (st != COSA_OK) return st;
+  const cosa_shape& s = *shape;
+  if (s.Nq != 1) return COSA_ESHAPE;
+  const int str = s.stride;
+  if (!pow2(str) || s.bk % str || s.bk / str > 32 || s.Nkv % str) return COSA_EUNSUPPORTED;
+  if (!(budget > 0.0) || budget > 1.0) return COSA_EINVAL;
+  const int nkb = n_kblocks(&s), nkp = s.Nkv / str;
+  if (nkb > 16384) return COSA_EUNSUPPORTED;
+  if ((long long)s.B * s.Hq == 0 || s.Nkv == 0) return COSA_OK;
+  if (!q || !k || !kp_cache || !order || !count || (s.paged && !page_table)) return COSA_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(kp_cache)) return COSA_EALIGN;
+  if (kp_capacity < nkp || kp_valid < 0 || kp_valid > nkp) return COSA_EINVAL;
+  if ((long long)s.B * s.Hkv * kp_capacity >= (1ll << 31)) return COSA_EUNSUPPORTED;
+  const int kk = budget_k(nkb, budget_bp(budget));
+  if (kmax < kk) return COSA_EINVAL;
+  if (decode_plan_smem(nkb, kk) > 227 * 1024) return COSA_EUNSUPPORTED;
+  // pool the keys no earlier call pooled into the cache
+  PoolParams pp;
+  pp.q = nullptr; pp.qp = nullptr;
+  pp.k = static_cast<const uint16_t*>(k);
+  pp.page_table = page_table;
+  pp.kp = static_cast<uint16_t*>(kp_cache);
+  pp.B = s.B; pp.Hq = s.Hq; pp.Hkv = s.Hkv; pp.Nq = s.Nq; pp.Nkv = s.Nkv; pp.s = str; pp.bk = s.bk;
+  pp.nkb = nkb; pp.paged = s.paged; pp.num_pages = s.num_pages;
+  pp.kp_first = kp_valid; pp.kp_stride = kp_capacity;
+  pp.q_items = 0;
+  pp.k_items = (long long)s.B * s.Hkv * (nkp - kp_valid);
+  if ((st = launch_status(launch_kap_pool(pp, stream))) != COSA_OK) return st;
+  DecodePlanParams dp;
+  dp.B = s.B; dp.Hq = s.Hq; dp.Hkv = s.Hkv;
+  dp.nkb = nkb; dp.nkp = nkp; dp.kpb = s.bk / str; dp.kp_stride = kp_capacity;
+  dp.k = kk; dp.kmax = kmax;
+  dp.q = static_cast<const uint16_t*>(q);
+  dp.kp = static_cast<const uint16_t*>(kp_cache);
+  dp.order = order; dp.count = count; dp.hrm_count = hrm_count;
+  dp.block_score = block_score; dp.hrm_flags = hrm_flags;
+  return launch_status(launch_decode_plan(dp, stream));
 }
 
 cosa_status cosa_block_union(const cosa_shape* shape, const int32_t* order, const int32_t* count, int kmax,

@@ -13,13 +13,10 @@
 // __syncwarp.  The row maxima come from kap_score's per-item partial maxima
 // (ties resolved to the smaller block index).  Each block's ranking key (+1
 // for HRM blocks, else its score <= 0) is mapped to an order-preserving
-// 32-bit integer.  A 4-pass, 8-bit radix select (per-warp shared-memory
-// histogram) finds the k-th largest value T; the blocks above T plus the
-// lowest-indexed blocks equal to T are compacted in index order with warp
-// ballots, and only those k keys -- packed with the inverted block index so
-// ties resolve to the smaller index -- are sorted by a bitonic network in
-// shared memory.
-#include "internal.h"
+// 32-bit integer, and warp_select_sort (kap_select.cuh: radix select of the
+// k-th key, ballot compaction, bitonic sort of the k kept keys) emits the
+// order.
+#include "kap_select.cuh"
 
 namespace cosa {
 
@@ -27,21 +24,9 @@ namespace {
 
 constexpr int kMaxWarps = 8;
 
-__device__ __forceinline__ uint32_t orderable(float f) {
-  const uint32_t u = __float_as_uint(f);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
 __device__ __forceinline__ int causal_blocks(int I, int Nq, int Nkv, int bq, int bk, int nkb) {
   const int last_tok = min((I + 1) * bq, Nq) - 1;
   return min(nkb, (Nkv - Nq + last_tok) / bk + 1);
-}
-
-__host__ __device__ __forceinline__ size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
-
-// Per-warp shared memory: a 256-bin histogram, the n keys, the P selected keys.
-__host__ __device__ __forceinline__ size_t warp_smem(int nkb, int pk) {
-  return 1024 + align16((size_t)nkb * 4) + (size_t)pk * 8;
 }
 
 template <int RPQ>
@@ -50,12 +35,11 @@ __global__ void __launch_bounds__(32 * kMaxWarps) kap_sort_kernel(SortParams p, 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * (blockDim.x >> 5) + warp;
   if (row >= rows) return;                       // whole warps only; no block-wide barrier below
-  uint8_t* mine = dyn + (size_t)warp * warp_smem(p.nkb, pk);
+  uint8_t* mine = dyn + (size_t)warp * select_smem(p.nkb, pk);
   int* hist = reinterpret_cast<int*>(mine);
   uint32_t* hi = reinterpret_cast<uint32_t*>(mine + 1024);
   uint64_t* sel = reinterpret_cast<uint64_t*>(mine + 1024 + align16((size_t)p.nkb * 4));
   const unsigned full = 0xffffffffu;
-  const unsigned lt_mask = (1u << lane) - 1u;
 
   const int I = row % p.nqb;
   const int hb = row / p.nqb;                    // b * Hq + h
@@ -119,99 +103,7 @@ __global__ void __launch_bounds__(32 * kMaxWarps) kap_sort_kernel(SortParams p, 
   for (int o = 16; o > 0; o >>= 1) hrm += __shfl_xor_sync(full, hrm, o);
   __syncwarp();
 
-  // ------------------------------------------------------------ radix select of the k-th largest
-  uint32_t T = 0;
-  int need = k;
-  if (k < n) {
-    uint32_t prefix = 0, mask = 0;
-    int remaining = k;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int b = lane; b < 256; b += 32) hist[b] = 0;
-      __syncwarp();
-      for (int i = lane; i < n; i += 32) {
-        const uint32_t h = hi[i];
-        if ((h & mask) == prefix) atomicAdd(&hist[(h >> shift) & 255u], 1);
-      }
-      __syncwarp();
-      // lane l owns digits 255-8l .. 248-8l (descending); counts from the top digit
-      int c[8], tot = 0;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) { c[q] = hist[255 - 8 * lane - q]; tot += c[q]; }
-      int incl = tot;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(full, incl, o);
-        if (lane >= o) incl += y;
-      }
-      const int excl = incl - tot;
-      const bool here = excl < remaining && remaining <= incl;
-      uint32_t digit = 0;
-      int rem_here = 0;
-      if (here) {
-        int acc = excl;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          if (acc + c[q] >= remaining) { digit = 255 - 8 * lane - q; rem_here = remaining - acc; break; }
-          acc += c[q];
-        }
-      }
-      const int src = __ffs(__ballot_sync(full, here)) - 1;
-      digit = __shfl_sync(full, digit, src);
-      remaining = __shfl_sync(full, rem_here, src);
-      prefix |= digit << shift;
-      mask |= 255u << shift;
-      __syncwarp();
-    }
-    T = prefix;
-    need = remaining;
-  }
-
-  // ------------------------------------------------------------ compaction in index order
-  const int total_gt = k - need;
-  int g = 0, e = 0;
-  for (int base = 0; base < n; base += 32) {
-    const int i = base + lane;
-    const uint32_t h = i < n ? hi[i] : 0u;
-    const uint64_t key = ((uint64_t)h << 32) | (uint64_t)(0xffffffffu - (uint32_t)i);
-    if (k == n) {
-      if (i < n) sel[i] = key;
-      continue;
-    }
-    const bool gt = i < n && h > T, eq = i < n && h == T;
-    const unsigned bg = __ballot_sync(full, gt), be = __ballot_sync(full, eq);
-    if (gt) sel[g + __popc(bg & lt_mask)] = key;
-    if (eq) {
-      const int r = e + __popc(be & lt_mask);
-      if (r < need) sel[total_gt + r] = key;
-    }
-    g += __popc(bg);
-    e += __popc(be);
-  }
-  int P = 1;
-  while (P < k) P <<= 1;
-  for (int i = k + lane; i < P; i += 32) sel[i] = 0;
-  __syncwarp();
-
-  // ------------------------------------------------------------ bitonic sort of the k keys, descending
-  for (int kk = 2; kk <= P; kk <<= 1) {
-    for (int j = kk >> 1; j > 0; j >>= 1) {
-      for (int i = lane; i < P; i += 32) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const uint64_t a = sel[i], b = sel[ixj];
-          const bool desc = (i & kk) == 0;
-          if (desc ? (a < b) : (a > b)) {
-            sel[i] = b;
-            sel[ixj] = a;
-          }
-        }
-      }
-      __syncwarp();
-    }
-  }
-  int32_t* ord = p.order + (size_t)row * p.kmax;
-  for (int t = lane; t < p.kmax; t += 32)
-    ord[t] = t < k ? (int32_t)(0xffffffffu - (uint32_t)(sel[t] & 0xffffffffu)) : -1;
+  warp_select_sort(hi, n, k, hist, sel, p.order + (size_t)row * p.kmax, p.kmax, lane);
   if (lane == 0) {
     p.count[row] = k;
     if (p.hrm_count) p.hrm_count[row] = hrm;
@@ -238,7 +130,7 @@ cudaError_t launch_kap_sort(const SortParams& p, cudaStream_t st) {
   if (rows == 0) return cudaSuccess;
   int pk = 1;
   while (pk < p.kmax) pk <<= 1;
-  const size_t per_warp = warp_smem(p.nkb, pk);
+  const size_t per_warp = select_smem(p.nkb, pk);
   int warps = (int)((96 * 1024) / per_warp);
   warps = warps < 1 ? 1 : (warps > kMaxWarps ? kMaxWarps : warps);
   const size_t smem = per_warp * warps;

@@ -134,6 +134,34 @@ COSA_API cosa_status cosa_plan_chunk(const cosa_shape* shape, const void* q, con
                                      void* workspace, size_t ws_bytes, uint32_t* dev_status,
                                      cudaStream_t stream);
 
+/* The Kernel-Aware Proxy for one decode step.  The CoSA pages treat only
+ * prefill and name decoding as future work (technical summary Sec. 4); this
+ * is the plainest single-row reading of Sec. 2.2: shape->Nq == 1, the query
+ * of each head sits at position Nkv - 1 and is not pooled, the keys are
+ * pooled as in prefill (mean of `stride` keys, kept in the caller's pooled-key
+ * cache exactly as for cosa_plan_chunk), and per head
+ *   S[c] = q . Kp[c] over every pooled key, MaxPool over each KV block's
+ *   pooled keys, MaxNorm (minus the maximum), HRM = the first block holding
+ *   the maximum, order = (HRM, score desc, block asc), the first
+ *   k = max(1, ceil(nKB * budget)) kept.
+ *  q          [B, Hq, 1, d] bf16 (16-byte aligned).
+ *  k          keys as for cosa_plan (contiguous or paged); rows kp_valid ..
+ *             Nkv/stride - 1 of kp_cache are pooled from it first.
+ *  kp_cache, kp_capacity, kp_valid: as for cosa_plan_chunk (Nkv must be a
+ *             multiple of stride).
+ *  order      [B, Hq, 1, kmax] int32 out (kmax >= k), padded -1; count,
+ *             hrm_count [B, Hq] out; block_score [B, Hq, nKB] fp32 and
+ *             hrm_flags [B, Hq, nKB] uint8 out (nullable).
+ * The decode step's attention is cosa_attend on the same shape (Nq = 1):
+ * with one valid row the tile-wide skip vote is that row's own test.
+ * Returns COSA_ESHAPE if Nq != 1, COSA_EINVAL for null pointers, a budget
+ * outside (0, 1], kp arguments out of range or kmax < k. */
+COSA_API cosa_status cosa_decode_plan(const cosa_shape* shape, const void* q, const void* k,
+                                      const int32_t* page_table, void* kp_cache, int kp_capacity, int kp_valid,
+                                      double budget, int kmax, int32_t* order, int32_t* count,
+                                      int32_t* hrm_count, float* block_score, uint8_t* hrm_flags,
+                                      cudaStream_t stream);
+
 /* Block union ("CompactAttention: Accelerating Chunked Prefill with
  * Block-Union KV Selection", method, selection stage): turn a per-head
  * selection into one KV block table per (batch, kv-head group), the union

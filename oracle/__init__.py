@@ -94,6 +94,71 @@ def block_union(wl, order: torch.Tensor, count: torch.Tensor):
     return tables, rows
 
 
+def decode_kap(q: torch.Tensor, k: torch.Tensor, bk: int, stride: int, budget: float):
+    """The Kernel-Aware Proxy for one decode step (CoSA technical summary
+    Sec. 2.2 with a single query row; the pages leave decoding to future
+    work, Sec. 4): the query of each head, at position Nkv-1, is not pooled
+    (a row of one token); the keys are pooled as in prefill (mean of
+    `stride` consecutive keys, bf16).  Scores S[c] = q . Kp[c] (all pooled
+    keys are visible to the last position), MaxPool over each block's pooled
+    keys, MaxNorm (minus the row max), HRM = first block holding the row max,
+    order = (HRM desc, score desc, block asc), k = max(1, ceil(nKB * bp /
+    1e4)).  Products are summed in fp64 and rounded to fp32 before every
+    comparison, like the prefill steps.
+    q [B, Hq, d] bf16; k logical [B, Hkv, Nkv, d] bf16 (Nkv a multiple of
+    stride).  Returns dict(order [B*Hq, k] int32, count [B*Hq], hrm_count,
+    score [B*Hq, nKB] fp32, hrm [B*Hq, nKB] uint8)."""
+    B, Hq, d = q.shape
+    Hkv, Nkv = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    nkb = -(-Nkv // bk)
+    kpb = bk // stride
+    kp = pool(k.reshape(B * Hkv * Nkv, d), stride).view(B, Hkv, Nkv // stride, d).double()
+    sc = torch.einsum("bhd,bhcd->bhc", q.double(), kp.repeat_interleave(G, dim=1)).float()
+    nkp = sc.shape[-1]
+    pad = nkb * kpb - nkp
+    bs = torch.nn.functional.pad(sc, (0, pad), value=float("-inf")).view(B, Hq, nkb, kpb).amax(-1)
+    bs = bs.reshape(B * Hq, nkb)
+    rowmax = bs.amax(-1, keepdim=True)
+    jstar = torch.argmax((bs == rowmax).to(torch.int8), dim=-1)      # first block holding the max
+    z = bs - rowmax                                                 # fp32 subtraction
+    hrm = torch.zeros_like(bs, dtype=torch.uint8)
+    hrm[torch.arange(B * Hq), jstar] = 1
+    bp = int(round(budget * 10000))
+    kk = max(1, min(nkb, -(-nkb * bp // 10000)))
+    order = torch.empty(B * Hq, kk, dtype=torch.int32)
+    for i in range(B * Hq):
+        keys = sorted(range(nkb), key=lambda j: (-int(hrm[i, j]), -float(z[i, j]), j))
+        order[i] = torch.tensor(keys[:kk], dtype=torch.int32)
+    return dict(order=order, count=torch.full((B * Hq,), kk, dtype=torch.int32),
+                hrm_count=hrm.sum(-1).to(torch.int32), score=z, hrm=hrm)
+
+
+def decode_osk(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, order: torch.Tensor, count: torch.Tensor,
+               bk: int, eps: float):
+    """The Ordered-Skipping Kernel for one decode step: OSK (Sec. 2.3) with a
+    single query row, so the tile-wide vote is that row's own test (no
+    bucket effect).  It is oracle_osk on the shape Nq = 1, bq = 1 (stride 1:
+    nothing is pooled here).  q [B, Hq, d]; k, v logical [B, Hkv, Nkv, d].
+    Returns osk()'s dict with out [B*Hq, 1, d]."""
+    B, Hq, d = q.shape
+    Hkv, Nkv = k.shape[1], k.shape[2]
+    sh = OrShape(B, Hq, Hkv, 1, Nkv, d, 1, bk, 1, 0, 0)
+    n = B * Hq
+    km = order.shape[1]
+    out = torch.empty(n, 1, d, dtype=torch.float64)
+    lse = torch.empty(n, 1, dtype=torch.float64)
+    skipped = torch.empty(n, km, dtype=torch.uint8)
+    margin = torch.empty(n, km, dtype=torch.float64)
+    qq = q.contiguous().view(B, Hq, 1, d)
+    rc = lib().oracle_osk(ctypes.byref(sh), _p(qq.view(torch.int16)), _p(k.contiguous().view(torch.int16)),
+                          _p(v.contiguous().view(torch.int16)), None, None, 0, _p(order.contiguous()),
+                          _p(count.contiguous()), km, eps, _p(out), _p(lse), _p(skipped), _p(margin), 0)
+    if rc != 0:
+        raise ValueError(f"oracle_osk failed ({rc})")
+    return dict(out=out, lse=lse, skipped=skipped, margin=margin)
+
+
 def shape_of(wl) -> OrShape:
     return OrShape(wl.B, wl.Hq, wl.Hkv, wl.Nq, wl.Nkv, wl.d, wl.bq, wl.bk, wl.stride,
                    1 if wl.paged else 0, wl.num_pages)

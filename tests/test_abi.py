@@ -134,6 +134,26 @@ def test_block_union_argument_errors_return_before_launch(cosa):
     assert call(shape=cosa.make_shape(0, 4, 2, 256, 768, 128, 128, 128, 16), table=None) == 0
 
 
+def test_decode_plan_argument_errors_return_before_launch(cosa):
+    lib = cosa._lib
+    s = cosa.make_shape(1, 4, 2, 1, 1024, 128, 128, 128, 16)        # one query after 1023 keys; nKB = 8
+    P = 1 << 20
+
+    def call(q=P, k=P, cache=P, cap=64, valid=0, budget=0.25, kmax=2, order=P, count=P, shape=s):
+        return lib.cosa_decode_plan(ctypes.byref(shape), q, k, None, cache, cap, valid, budget, kmax, order,
+                                    count, None, None, None, None)
+    assert call(shape=cosa.make_shape(1, 4, 2, 2, 1024, 128, 128, 128, 16)) == 3     # Nq != 1
+    assert call(shape=cosa.make_shape(1, 4, 2, 1, 1000, 128, 128, 128, 16)) == 6     # Nkv not a stride multiple
+    assert call(cache=None) == 1
+    assert call(q=None) == 1
+    assert call(budget=0.0) == 1
+    assert call(kmax=1) == 1                      # ceil(8 * 0.25) = 2 blocks kept
+    assert call(cap=63) == 1
+    assert call(valid=65) == 1
+    assert call(q=P + 4) == 2
+    assert call(shape=cosa.make_shape(0, 4, 2, 1, 1024, 128, 128, 128, 16), q=None) == 0
+
+
 def test_attend_argument_errors_return_before_launch(cosa):
     lib = cosa._lib
     s = cosa.make_shape(1, 4, 2, 256, 512, 128, 128, 64, 16)

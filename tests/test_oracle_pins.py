@@ -521,3 +521,81 @@ def test_block_union_properties_random():
                 for I in range(wl.n_qblocks):
                     last_key = off + min((I + 1) * wl.bq, wl.Nq) - 1
                     assert rows[(b * wl.Hq + h) * wl.n_qblocks + I] == [j for j in tab if j * wl.bk <= last_key]
+
+
+# ----------------------------------------------------------------- decode step
+
+@pytest.mark.parametrize("bk", [64, 128])
+def test_decode_kap_equals_prefill_kap_of_a_repeated_query(bk):
+    """A decode query at position Nkv-1 is the prefill proxy's single pooled
+    row when its Q-block holds 16 copies of that query: the mean of 16 equal
+    bf16 values is the value itself, the pooled causality 16c <= off + 15
+    admits every pooled key, and the budget counts every block.  So the
+    Python decode proxy must agree exactly with the C prefill proxy there."""
+    g = torch.Generator().manual_seed(5)
+    B, Hq, Hkv, Nkv, d = 2, 4, 2, 1024 + 3 * bk, 32
+    q = (torch.randn(B, Hq, d, generator=g) * 2).to(torch.bfloat16)
+    k = torch.randn(B, Hkv, Nkv, d, generator=g).to(torch.bfloat16)
+    k[:, :, 5 * bk + 7] += 6                                        # a clear maximum somewhere
+    for budget in (0.1, 0.37, 1.0):
+        dec = oracle.decode_kap(q, k, bk, 16, budget)
+        wl = tiny(B=B, Hq=Hq, Hkv=Hkv, Nq=16, Nkv=Nkv, d=d, bq=16, bk=bk)
+        qq = q[:, :, None, :].expand(B, Hq, 16, d).contiguous()
+        inp = synth.Inputs(wl, qq, k.contiguous(), k.contiguous())
+        ref = oracle.kap(inp, budget, want_scores=True)
+        assert torch.equal(dec["order"], ref["order"][:, : dec["order"].shape[1]])
+        assert torch.equal(dec["count"], ref["count"])
+        assert torch.equal(dec["hrm_count"], ref["hrm_count"])
+        assert torch.equal(dec["score"], ref["score"])
+        assert torch.equal(dec["hrm"], ref["hrm"])
+
+
+def test_decode_osk_eps0_is_dense_attention_of_the_row():
+    """With eps = 0 nothing is skipped, and visiting every block in any order
+    is softmax attention of the one query row over the whole cache
+    (Sec. 2.1, order invariance), checked against torch's SDPA in fp64."""
+    g = torch.Generator().manual_seed(6)
+    B, Hq, Hkv, Nkv, d, bk = 1, 4, 2, 1000, 128, 128
+    q = torch.randn(B, Hq, d, generator=g).to(torch.bfloat16)
+    k = torch.randn(B, Hkv, Nkv, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, Hkv, Nkv, d, generator=g).to(torch.bfloat16)
+    nkb = -(-Nkv // bk)
+    order = torch.stack([torch.randperm(nkb, generator=g) for _ in range(B * Hq)]).to(torch.int32)
+    count = torch.full((B * Hq,), nkb, dtype=torch.int32)
+    res = oracle.decode_osk(q, k, v, order, count, bk, 0.0)
+    kk = k.double().repeat_interleave(Hq // Hkv, dim=1)
+    vv = v.double().repeat_interleave(Hq // Hkv, dim=1)
+    ref = torch.nn.functional.scaled_dot_product_attention(q.double()[:, :, None, :], kk, vv)
+    assert torch.allclose(res["out"].view(B, Hq, 1, d), ref, atol=1e-12, rtol=1e-10)
+    assert int(res["skipped"].sum()) == 0
+
+
+def test_decode_osk_skip_is_the_rows_own_test():
+    """With one row the tile-wide vote is the row's own test: on integer
+    logits, a visited block is skipped exactly when its max minus the running
+    max (over the computed blocks before it) is below T, computed here by
+    brute force."""
+    g = torch.Generator().manual_seed(7)
+    B, Hq, Hkv, Nkv, d, bk = 1, 2, 1, 1024, 32, 64
+    q = torch.randint(-2, 3, (B, Hq, d), generator=g).to(torch.bfloat16)
+    k = torch.randint(-2, 3, (B, Hkv, Nkv, d), generator=g).to(torch.bfloat16)
+    k[:, :, 130] += 4 * q[:, 0].sign().to(torch.bfloat16)           # a block with much larger logits
+    v = torch.randint(-2, 3, (B, Hkv, Nkv, d), generator=g).to(torch.bfloat16)
+    nkb = Nkv // bk
+    order = torch.stack([torch.tensor([2] + [j for j in range(nkb) if j != 2])] * Hq).to(torch.int32)
+    count = torch.full((Hq,), nkb, dtype=torch.int32)
+    eps = 1e-3
+    res = oracle.decode_osk(q, k, v, order, count, bk, eps)
+    T = oracle.skip_threshold(eps, d)
+    for h in range(Hq):
+        logits = (q[0, h].double() @ k[0, 0].double().T)
+        m_run = float("-inf")
+        for t in range(nkb):
+            j = int(order[h, t])
+            m_loc = float(logits[j * bk:(j + 1) * bk].max())
+            skip = m_run != float("-inf") and (torch.tensor(m_loc, dtype=torch.float32) -
+                                               torch.tensor(m_run, dtype=torch.float32)).item() < T
+            assert int(res["skipped"][h, t]) == int(skip), (h, t)
+            if not skip:
+                m_run = max(m_run, m_loc)
+    assert int(res["skipped"].sum()) > 0
