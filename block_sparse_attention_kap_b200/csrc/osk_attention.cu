@@ -27,6 +27,9 @@
 // [0, BK), O at [128, 256); 256 columns and ~104 KB of shared memory per
 // CTA, so two CTAs share an SM and one CTA's softmax overlaps the other's
 // tensor-core work.
+// The softmax warps are bound by instruction issue (with the MUFU pipe a
+// close second), so pass 1 takes maxima three at a time and pass 2 forms the
+// exponent arguments and the row sums with packed f32x2 arithmetic.
 #include <cuda_bf16.h>
 #include "internal.h"
 #include "sm100.cuh"
@@ -80,6 +83,31 @@ __device__ __forceinline__ bool all_rows(bool v) {
       : "r"((uint32_t)v)
       : "memory");
   return r != 0;
+}
+
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void up2(uint64_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -217,18 +245,19 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                    desc_sw128(slot_addr(ks) + kk * 2048, Cfg::kChunk, 1024), id_pv, (any_pv || kk > 0) ? 1u : 0u);
           any_pv = true;
           if (t + 2 < n) pend_k = t + 2;
-        } else if (t + 2 < n) {
-          // a skipped block's S was fully read before the vote: the next QK may
-          // overwrite it at once (p_ready of this visit completes before the
-          // next vote, so its phase parity stays in step)
-          load(ks, &tm_k, order_at(t + 2));
         }
+        // a skipped block's S was fully read before the vote: the next QK may
+        // overwrite it at once (p_ready of this visit completes before the
+        // next vote, so its phase parity stays in step); its slot then takes
+        // K of visit t + 2, issued after that QK so the QK is not delayed
         if (t + 1 < n) {
           if (!wait_slot(ns)) break;
           tc_fence_after();
           issue_qk(ns);
         }
+        if (dec != kDecisionCompute && t + 2 < n) load(ks, &tm_k, order_at(t + 2));
         ks = ns;
+
       }
       // o_final completes once every MMA issued above has; TMEM is released after it
       tc_commit(&sm->o_final);
@@ -266,7 +295,7 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         tmem_ld_x64(tS + lane_base + c_base, v);
         if (lim >= c_base + 63) {
 #pragma unroll
-          for (int i = 0; i < 64; ++i) mp[i & 3] = fmaxf(mp[i & 3], __uint_as_float(v[i]));
+          for (int i = 0; i < 32; ++i) mp[i & 3] = max3f(mp[i & 3], __uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
         } else {
 #pragma unroll
           for (int i = 0; i < 64; ++i) mp[i & 3] = fmaxf(mp[i & 3], c_base + i <= lim ? __uint_as_float(v[i]) : -INFINITY);
@@ -311,7 +340,8 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         // TMEM columns [c_base, c_base + HC/2): inside this half's own S range
         // and behind its reads, so the other half's S is never overwritten
         const float msl = (m_scale == -INFINITY) ? 0.0f : m_scale * sl2;
-        float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        uint64_t ls2[2] = {0ull, 0ull};           // packed partial row sums
+        const uint64_t sl2x2 = pk2(sl2, sl2), nmsl2 = pk2(-msl, -msl);
 #pragma unroll 1
         for (int c0 = c_base; c0 < c_base + HC; c0 += 16) {
           uint32_t v[16];
@@ -324,14 +354,20 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           uint32_t w[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const float p0 = ex2(fmaf(__uint_as_float(v[2 * i]), sl2, -msl));
-            const float p1 = ex2(fmaf(__uint_as_float(v[2 * i + 1]), sl2, -msl));
-            ls[i & 3] += p0 + p1;
+            float x0, x1;
+            up2(fma2(pk2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), sl2x2, nmsl2), x0, x1);
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            ls2[i & 1] = add2(ls2[i & 1], pk2(p0, p1));
             w[i] = pack_bf16(p0, p1);
           }
           tmem_st_x8(tS + lane_base + c_base + (c0 - c_base) / 2, w);
         }
-        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        {
+          float a0, a1, b0, b1;
+          up2(ls2[0], a0, a1);
+          up2(ls2[1], b0, b1);
+          l += (a0 + b0) + (a1 + b1);
+        }
         // rescale this half of O when the exponent reference moved
         if (any_pv && __any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll 1
