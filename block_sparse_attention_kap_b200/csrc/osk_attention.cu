@@ -336,32 +336,33 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         }
         l *= alpha;
         // pass 2: P = exp2((S - m_scale) * log2(e)/sqrt(d)) over this half's
-        // columns, re-read 16 at a time and written back as bf16 pairs into
+        // columns, re-read 32 at a time and written back as bf16 pairs into
         // TMEM columns [c_base, c_base + HC/2): inside this half's own S range
         // and behind its reads, so the other half's S is never overwritten
         const float msl = (m_scale == -INFINITY) ? 0.0f : m_scale * sl2;
         uint64_t ls2[2] = {0ull, 0ull};           // packed partial row sums
         const uint64_t sl2x2 = pk2(sl2, sl2), nmsl2 = pk2(-msl, -msl);
 #pragma unroll 1
-        for (int c0 = c_base; c0 < c_base + HC; c0 += 16) {
-          uint32_t v[16];
-          tmem_ld_x16(tS + lane_base + c0, v);
-          if (lim < c0 + 15) {
+        for (int c0 = c_base; c0 < c_base + HC; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld_x32(tS + lane_base + c0, v);
+          if (lim < c0 + 31) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
+            for (int i = 0; i < 32; ++i)
               if (c0 + i > lim) v[i] = __float_as_uint(-INFINITY);
           }
-          uint32_t w[8];
+          uint32_t w[16];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
+          for (int i = 0; i < 16; ++i) {
             float x0, x1;
             up2(fma2(pk2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), sl2x2, nmsl2), x0, x1);
             const float p0 = ex2(x0), p1 = ex2(x1);
             ls2[i & 1] = add2(ls2[i & 1], pk2(p0, p1));
             w[i] = pack_bf16(p0, p1);
           }
-          tmem_st_x8(tS + lane_base + c_base + (c0 - c_base) / 2, w);
+          tmem_st_x16(tS + lane_base + c_base + (c0 - c_base) / 2, w);
         }
+
         {
           float a0, a1, b0, b1;
           up2(ls2[0], a0, a1);
