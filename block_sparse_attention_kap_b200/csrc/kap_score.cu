@@ -169,24 +169,29 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
       const int c_lo = T * kTileRows + 64 * half;              // first pooled key of this half
       // a half every column of which this row sees needs no per-column test
       const bool full = got && row_ok && c_lo + 63 <= climit && c_lo + 64 <= p.nkp;
-#pragma unroll
-      for (int qc = 0; qc < 2; ++qc) {
-        uint32_t v[32];
-        tmem_ld_x32(tmem_addr(tmem, 32 * quarter, st * 128 + 64 * half + 32 * qc), v);
+      {
+        uint32_t v[64];
+        tmem_ld_x64(tmem_addr(tmem, 32 * quarter, st * 128 + 64 * half), v);
+        // the accumulator stage is in registers: hand it back to the MMA at once
+        tc_fence_before();
+        mbar_arrive(&sm->s_free[st]);
         if (full) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) bsv[(32 * qc + i) / KPB] = fmaxf(bsv[(32 * qc + i) / KPB], __uint_as_float(v[i]));
+          for (int i = 0; i < 64; i += 2) {
+            float m3;
+            asm("max.f32 %0, %1, %2, %3;" : "=f"(m3) : "f"(bsv[i / KPB]), "f"(__uint_as_float(v[i])), "f"(__uint_as_float(v[i + 1])));
+            bsv[i / KPB] = m3;
+          }
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int c = c_lo + 32 * qc + i;
+          for (int i = 0; i < 64; ++i) {
+            const int c = c_lo + i;
             const bool vis = got && row_ok && c <= climit && c < p.nkp;
-            bsv[(32 * qc + i) / KPB] = fmaxf(bsv[(32 * qc + i) / KPB], vis ? __uint_as_float(v[i]) : -INFINITY);
+            bsv[i / KPB] = fmaxf(bsv[i / KPB], vis ? __uint_as_float(v[i]) : -INFINITY);
           }
         }
       }
-      tc_fence_before();
-      mbar_arrive(&sm->s_free[st]);
+
       const int j0 = T * BPT + half * BPH;                     // first block of this half
 #pragma unroll
       for (int jh = 0; jh < BPH; ++jh)
