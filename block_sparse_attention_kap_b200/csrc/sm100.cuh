@@ -92,7 +92,7 @@ __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
 }
 
 // ------------------------------------------------------------------ TMA
-// 2D tiled load, completion signalled on an mbarrier (no multicast).
+// 2D tiled load into this CTA's shared memory, completion signalled on an mbarrier.
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"

@@ -1,6 +1,6 @@
 """Parity of the CUDA path (through the C ABI) against the CPU oracle.
 
-Bar (the benchmark spec): M_KAP (order, count, HRM) and the in-kernel skip
+Bar: M_KAP (order, count, HRM) and the in-kernel skip
 decisions bit-exact on integer-grid inputs, where every pooled value and
 logit is exact; outputs within max-abs 1e-2 of the exact result (plus one
 bf16 half-ulp of the value, since |out| >= 4 has a bf16 spacing above 2e-2)
