@@ -6,7 +6,12 @@ never imports, calls or links it.
 
 Every function takes host torch tensors (bf16 inputs as produced by
 ``synth``) and returns host tensors.  Semantics: see cosa_oracle.c; each
-step cites the CoSA technical summary (Sec. 2.1-2.3).
+step cites the CoSA technical summary (Sec. 2.1-2.3).  Beyond the C
+library: ``block_union`` (CompactAttention's selection stage, Python sets),
+``decode_kap`` / ``decode_osk`` (one decode step: the single-row reading of
+Sec. 2.2/2.3), ``round_bf16`` (fp64 -> nearest bf16).  All are pinned in
+tests/test_oracle_pins.py against hand-worked examples, independent
+formulations (the C prefill proxy, torch SDPA, brute force) or properties.
 """
 from __future__ import annotations
 
