@@ -375,3 +375,57 @@ def test_edge_shapes_bit_exact(cosa, shape, budget, eps):
     o = oracle.osk(inp, ref["order"], ref["count"], eps)
     assert torch.equal(cosa.unpack_skip_bits(flat(res["skip_bits"]), km), o["skipped"])
     check_out(gpu_rows(res["out"], wl), o["out"])
+
+
+def test_visit_list_longer_than_the_staged_order(cosa):
+    """One Q-block visiting 1,280 KV blocks (64-key blocks of an 81,920-token
+    cache): the kernel stages the first 1,024 order entries in shared memory
+    and reads the rest from global memory; dense (eps 0) and eps > 0 both
+    match the oracle, skip bits included (integer grid, structured)."""
+    wl = tiny(Hq=1, Hkv=1, Nq=128, Nkv=81920, bq=128, bk=64, structured=True, n_needle=2)
+    inp = synth.generate(wl, grid=True)
+    m = cosa.CoSA(cosa.shape_of_workload(wl))
+    q, k, v = inp.q.cuda(), inp.k.cuda(), inp.v.cuda()
+    assert m.nkb == 1280
+    g = torch.Generator().manual_seed(12)
+    order = torch.randperm(m.nkb, generator=g).to(torch.int32).view(1, 1, 1, -1)
+    count = torch.full((1, 1, 1), m.nkb, dtype=torch.int32)
+    for eps in (0.0, EPS):
+        res = m.attend(q, k, v, order.cuda(), count.cuda(), eps, lse=True, skip_bits=True)
+        torch.cuda.synchronize()
+        assert m.device_status() == 0
+        o = oracle.osk(inp, order.view(1, -1), count.view(-1), eps)
+        bits = cosa.unpack_skip_bits(flat(res["skip_bits"]), m.nkb)
+        assert torch.equal(bits, o["skipped"])
+        if eps > 0:
+            assert int(bits[0, 1024:].sum()) > 0          # decisions past the staged part
+        check_out(gpu_rows(res["out"], wl), o["out"])
+
+
+STRIDE_SHAPES = [
+    dict(Hq=2, Hkv=1, Nq=512, Nkv=1024, bq=128, bk=128, stride=4),      # 32 pooled rows per Q-block, 32 keys per block
+    dict(Hq=2, Hkv=2, Nq=768, Nkv=768, bq=128, bk=64, stride=8),        # 16 rows per Q-block, 8 keys per block
+    dict(Hq=4, Hkv=2, Nq=512, Nkv=1536, bq=64, bk=128, stride=32),      # 2 rows per Q-block, 4 keys per block
+]
+
+
+@pytest.mark.parametrize("shape", STRIDE_SHAPES)
+def test_other_pooling_strides_bit_exact(cosa, shape):
+    """Pooling strides other than 16 (every row-per-Q-block and key-per-block
+    count the kernels instantiate): plans and skip bits bit-exact on
+    structured grids, outputs within tolerance."""
+    kw = dict(shape)
+    stride = kw.pop("stride")
+    wl = tiny(structured=True, n_needle=2, stride=stride, **kw)
+    inp = synth.generate(wl, grid=True)
+    m, dev, plan = gpu_plan(cosa, inp, 0.4)
+    ref = oracle.kap(inp, 0.4, want_scores=True)
+    km = ref["order"].shape[1]
+    assert torch.equal(flat(plan["order"])[:, :km], ref["order"])
+    assert torch.equal(flat(plan["count"]).view(-1), ref["count"])
+    assert torch.equal(flat(plan["block_score"]), ref["score"])
+    assert torch.equal(flat(plan["hrm"]), ref["hrm"])
+    res = gpu_attend(m, dev, plan["order"], plan["count"], EPS)
+    o = oracle.osk(inp, ref["order"], ref["count"], EPS)
+    assert torch.equal(cosa.unpack_skip_bits(flat(res["skip_bits"]), km), o["skipped"])
+    check_out(gpu_rows(res["out"], wl), o["out"])
