@@ -290,7 +290,7 @@ class CoSA:
                     stream=None):
         """The proxy for one decode step (shape.Nq == 1)."""
         s = self.shape
-        km = max(cosa_kmax_decode(s, budget), 1)
+        km = self.nkb                      # row stride of order: room for every block; count says how many
         order = torch.empty(s.B, s.Hq, 1, km, dtype=torch.int32, device=self.device)
         count = torch.empty(s.B, s.Hq, 1, dtype=torch.int32, device=self.device)
         hrm = torch.empty(s.B, s.Hq, 1, dtype=torch.int32, device=self.device)
@@ -343,13 +343,6 @@ class CoSA:
 
     def device_status(self) -> int:
         return int(self.status.item())
-
-
-def cosa_kmax_decode(shape: cosa_shape, budget: float) -> int:
-    """Blocks a decode step keeps: max(1, ceil(nKB * round(budget * 1e4) / 1e4))."""
-    nkb = cosa_num_kblocks(shape)
-    bp = int(round(budget * 10000))
-    return max(1, min(nkb, -(-nkb * bp // 10000)))
 
 
 def shape_of_workload(wl) -> cosa_shape:
