@@ -567,6 +567,28 @@ def main():
                  "frac_of_peak": dense_flops / (dense_ms * 1e-3) / 1e12 / tc_peak,
                  "speedup_of_sparse_step": dense_ms / ms_step}
         del d_order, d_count
+        # context only, not this library: torch's fused causal attention on the
+        # same inputs (whatever backend torch picks), when its top-left causal
+        # alignment matches (Nq == Nkv) and K/V are contiguous
+        if wl.Nq == wl.Nkv and not wl.paged:
+            try:
+                sdpa = torch.nn.functional.scaled_dot_product_attention
+                o_ref = sdpa(q, k, v, is_causal=True, enable_gqa=True)
+                torch.cuda.synchronize()
+                a, b = ev(), ev()
+                a.record(stream)
+                for _ in range(dsteps):
+                    o_ref = sdpa(q, k, v, is_causal=True, enable_gqa=True)
+                b.record(stream)
+                torch.cuda.synchronize()
+                sdpa_ms = max_over_ranks([a.elapsed_time(b) / dsteps], dist, dev)[0]
+                dense["torch_sdpa_context"] = {
+                    "ms": sdpa_ms, "tflops": dense_flops / (sdpa_ms * 1e-3) / 1e12,
+                    "speedup_of_sparse_step": sdpa_ms / ms_step,
+                    "note": "torch.nn.functional.scaled_dot_product_attention, library kernel, context only"}
+                del o_ref
+            except (RuntimeError, TypeError) as exc:
+                dense["torch_sdpa_context"] = {"unavailable": str(exc).splitlines()[0][:200]}
 
     # ---------------------------------------------------------- end to end through the public API (host buffers)
     # Every step copies its inputs from pinned host memory and its output
