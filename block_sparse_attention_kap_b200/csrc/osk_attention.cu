@@ -360,8 +360,9 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             ls2[i & 1] = add2(ls2[i & 1], pk2(p0, p1));
             w[i] = pack_bf16(p0, p1);
           }
-          tmem_st_x16(tS + lane_base + c_base + (c0 - c_base) / 2, w);
+          tmem_st_x16_nowait(tS + lane_base + c_base + (c0 - c_base) / 2, w);
         }
+        tmem_wait_st();                           // every P store of this half is in TMEM
 
         {
           float a0, a1, b0, b1;
