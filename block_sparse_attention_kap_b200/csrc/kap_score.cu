@@ -113,20 +113,26 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
       tma_load_2d(sQ, &tm_qp, &sm->q_full, 0, qp_y);
       tma_load_2d(sQ + 16384, &tm_qp, &sm->q_full, 64, qp_y);
     }
+    uint32_t busy = 0u;    // stage bits: a key-tile load issued and not yet seen complete
+    uint32_t kph = 0u;     // stage bits: parity of the next completion on that stage
     for (int u = 0; u < 2 && u < U; ++u) {
       uint8_t* dst = sK + u * kTileBytes;
       const int y = kp_y0 + (t0 + u) * kTileRows;
+      busy |= 1u << u;
       mbar_arrive_expect_tx(&sm->k_full[u], kTileBytes);
       tma_load_2d(dst, &tm_kp, &sm->k_full[u], 0, y);
       tma_load_2d(dst + 16384, &tm_kp, &sm->k_full[u], 64, y);
     }
-    bool ok = U > 0 && wait_or_abort(&sm->q_full, 0, abort, p.status, DEV_TIMEOUT_TMA);
+    const bool q_seen = U > 0 && wait_or_abort(&sm->q_full, 0, abort, p.status, DEV_TIMEOUT_TMA);
+    bool ok = q_seen;
     const uint32_t idesc = idesc_bf16(128, 128, false, false);
     const uint32_t q_addr = smem_u32(sQ);
     for (int u = 0; ok && u < U; ++u) {
       const int st = u & 1;
       const uint32_t ph = (u >> 1) & 1;
       if (!wait_or_abort(&sm->k_full[st], ph, abort, p.status, DEV_TIMEOUT_TMA)) break;
+      busy &= ~(1u << st);
+      kph ^= 1u << st;
       if (u >= 2 && !wait_or_abort(&sm->s_free[st], ((u >> 1) - 1) & 1, abort, p.status, DEV_TIMEOUT_PIPE)) break;
       tc_fence_after();
       const uint32_t k_addr = smem_u32(sK + st * kTileBytes);
@@ -139,6 +145,7 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
         if (!wait_or_abort(&sm->s_full[st], ph, abort, p.status, DEV_TIMEOUT_MMA)) break;
         uint8_t* dst = sK + st * kTileBytes;
         const int y = kp_y0 + (t0 + u + 2) * kTileRows;
+        busy |= 1u << st;
         mbar_arrive_expect_tx(&sm->k_full[st], kTileBytes);
         tma_load_2d(dst, &tm_kp, &sm->k_full[st], 0, y);
         tma_load_2d(dst + 16384, &tm_kp, &sm->k_full[st], 64, y);
@@ -147,6 +154,12 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
     // every MMA this thread issued has completed before TMEM is released
     tc_commit(&sm->drained);
     mbar_wait(&sm->drained, 0);
+    // no copy may still be writing shared memory when the CTA exits: after a
+    // failed wait, wait again (bounded) for the loads not yet seen complete
+    // (one per stage at most; none on the normal path)
+    if (U > 0 && !q_seen) mbar_wait(&sm->q_full, 0);
+    for (int st = 0; st < 2; ++st)
+      if (busy & (1u << st)) mbar_wait(&sm->k_full[st], (kph >> st) & 1u);
   } else if (warp < kEpiWarps) {
     // ------------------------------------------------ epilogue: one pooled row, one column half
     const int quarter = warp & 3, half = warp >> 2;

@@ -196,15 +196,20 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       auto slot = [&](int sl) { return sl ? sV : sK; };
       auto slot_addr = [&](int sl) { return sl ? v_addr : k_addr; };
       uint32_t fph = 0u;     // bit sl: parity of the next completion to wait for on slot sl
+      uint32_t busy = 0u;    // bit sl: a load into slot sl was issued and not yet seen complete
       auto load = [&](int sl, const CUtensorMap* tm, int j) {
         const int y = kv_row<BK>(p, b, g, j);
+        busy |= 1u << sl;
         mbar_arrive_expect_tx(&sm->full[sl], Cfg::kKVBytes);
         tma_load_2d(slot(sl), tm, &sm->full[sl], 0, y);
         tma_load_2d(slot(sl) + Cfg::kChunk, tm, &sm->full[sl], 64, y);
       };
       auto wait_slot = [&](int sl) {
         const bool r = wait_or_abort(&sm->full[sl], (fph >> sl) & 1u, abort, p.status, DEV_TIMEOUT_TMA);
-        fph ^= 1u << sl;
+        if (r) {
+          fph ^= 1u << sl;
+          busy &= ~(1u << sl);
+        }
         return r;
       };
       auto issue_qk = [&](int sl) {
@@ -220,7 +225,8 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       load(0, &tm_k, order_at(0));
       if (n > 1) load(1, &tm_k, order_at(1));
       bool any_pv = false;
-      bool ok = wait_or_abort(&sm->q_full, 0, abort, p.status, DEV_TIMEOUT_TMA) && wait_slot(0);
+      const bool q_seen = wait_or_abort(&sm->q_full, 0, abort, p.status, DEV_TIMEOUT_TMA);
+      bool ok = q_seen && wait_slot(0);
       if (ok) { tc_fence_after(); issue_qk(0); }
       int ks = 0;            // slot holding K of visit t
       int pend_k = -1;       // K load deferred until the PV reading its slot has completed
@@ -262,6 +268,12 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       // o_final completes once every MMA issued above has; TMEM is released after it
       tc_commit(&sm->o_final);
       mbar_wait(&sm->o_final, 0);
+      // no copy may still be writing shared memory when the CTA exits: after a
+      // failed wait, wait again (bounded) for the loads not yet seen complete
+      // (a slot holds at most one outstanding load; none on the normal path)
+      if (!q_seen) mbar_wait(&sm->q_full, 0);
+      for (int sl = 0; sl < 2; ++sl)
+        if (busy & (1u << sl)) mbar_wait(&sm->full[sl], (fph >> sl) & 1u);
     }
   } else if (warp < kSoftmaxThreads / 32) {
     // ------------------------------------------------------------ softmax: one row, one column half
