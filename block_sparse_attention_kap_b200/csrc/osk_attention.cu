@@ -27,9 +27,13 @@
 // [0, BK), O at [128, 256); 256 columns and ~104 KB of shared memory per
 // CTA, so two CTAs share an SM and one CTA's softmax overlaps the other's
 // tensor-core work.
-// The softmax warps are bound by instruction issue (with the MUFU pipe a
-// close second), so pass 1 takes maxima three at a time and pass 2 forms the
-// exponent arguments and the row sums with packed f32x2 arithmetic.
+// Each CTA is one dependency chain per visit -- QK, the max and the vote,
+// the exponentials, PV, the next QK (S and P share TMEM columns) -- and no
+// single pipe is saturated: the chain's latency sets the pace, and the
+// second CTA on the SM fills part of it.  Pass 1 takes maxima three at a
+// time and pass 2 forms the exponent arguments and row sums with packed
+// f32x2 arithmetic and stores P without waiting per store, to shorten the
+// softmax's share of the chain.
 #include <cuda_bf16.h>
 #include "internal.h"
 #include "sm100.cuh"
