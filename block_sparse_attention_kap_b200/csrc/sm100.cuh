@@ -66,7 +66,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // limit_ns nanoseconds.  Returns false on timeout (the caller reports it and
 // unwinds); no wait in these kernels is unbounded.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = 1000000000ull) {
-  if (mbar_try_wait(bar, parity)) return true;
+  // the timer is read only after the phase has kept the thread waiting for
+  // a while, so a wait that ends soon never pays for a timer read
+  for (int i = 0; i < 64; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
