@@ -7,8 +7,6 @@ import hashlib
 import json
 import os
 
-import pytest
-
 import bench
 
 
