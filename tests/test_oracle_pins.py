@@ -13,6 +13,7 @@ import random
 
 import numpy as np
 import pytest
+from hypothesis import given, settings, strategies as st
 import torch
 
 import oracle
@@ -248,6 +249,33 @@ def test_kap_exact_on_grid(shape, beta):
             assert res["score"][i, j].item() == z / s2
             assert res["hrm"][i, j].item() == hrm[j]
         assert res["hrm_count"][i].item() == sum(hrm.values())
+
+
+@settings(max_examples=30, deadline=None, derandomize=True)
+@given(B=st.sampled_from([1, 2]), hq_g=st.sampled_from([(1, 1), (2, 1), (2, 2), (4, 2), (4, 4)]),
+       bq=st.sampled_from([32, 64, 128]), bk=st.sampled_from([32, 64, 128]), stride=st.sampled_from([8, 16]),
+       nq_units=st.integers(1, 24), off_units=st.integers(0, 24), beta=st.sampled_from([0.05, 0.3, 0.7, 1.0]),
+       structured=st.booleans(), wid=st.integers(0, 500))
+def test_kap_exact_on_random_grids(B, hq_g, bq, bk, stride, nq_units, off_units, beta, structured, wid):
+    """The same integer-exact brute force over random shapes: ragged Q- and
+    KV-blocks, a causal offset (queries after a cache), strides 8 and 16,
+    GQA groups of 1-4 heads and budgets from 5% to 100%."""
+    Hq, G = hq_g
+    Nq = stride * nq_units
+    Nkv = Nq + stride * off_units
+    wl = tiny(d=16, wid=wid, B=B, Hq=Hq, Hkv=Hq // G, Nq=Nq, Nkv=Nkv, bq=bq, bk=bk, stride=stride,
+              structured=structured, n_needle=1 if structured else 0)
+    inp = synth.generate(wl, grid=True)
+    res = oracle.kap(inp, beta, want_scores=True)
+    ref = _exact_kap(wl, inp.q.float(), inp.k.float(), beta)
+    s2 = float(stride ** 2)
+    for (b, h, I), (ordr, score, hrm) in ref.items():
+        i = (b * wl.Hq + h) * wl.n_qblocks + I
+        assert res["count"][i].item() == len(ordr)
+        assert res["order"][i, : len(ordr)].tolist() == ordr
+        for j, z in score.items():
+            assert res["score"][i, j].item() == z / s2
+            assert res["hrm"][i, j].item() == hrm[j]
 
 
 # ----------------------------------------------------------------- KAP: invariants on real-valued data
