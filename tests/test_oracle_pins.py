@@ -464,6 +464,46 @@ def test_skip_decisions_bruteforce_grid():
     assert res["skipped"].sum().item() > 0          # decisions of both kinds were checked
 
 
+@settings(max_examples=25, deadline=None, derandomize=True)
+@given(hq_g=st.sampled_from([(1, 1), (2, 1), (4, 2)]), bq=st.sampled_from([32, 64]), bk=st.sampled_from([32, 64]),
+       nq_units=st.integers(1, 12), off_units=st.integers(0, 12), frac=st.sampled_from([0.3, 0.7, 1.0]),
+       eps=st.sampled_from([1e-4, 1e-3, 0.05, 0.5]), wid=st.integers(0, 500))
+def test_skip_decisions_bruteforce_random(hq_g, bq, bk, nq_units, off_units, frac, eps, wid):
+    """The same definition over random shapes and visit orders: ragged last
+    Q-block (rows past Nq take no part in the vote), queries after a cache,
+    GQA groups, random subsets of the causal blocks in random order."""
+    Hq, G = hq_g
+    Nq = 16 * nq_units
+    Nkv = Nq + 16 * off_units
+    wl = tiny(d=32, wid=wid, Hq=Hq, Hkv=Hq // G, Nq=Nq, Nkv=Nkv, bq=bq, bk=bk, structured=True, n_needle=1)
+    inp = synth.generate(wl, grid=True)
+    order, count, _ = _random_orders(wl, frac, wid)
+    T = math.log(eps) * math.sqrt(wl.d)
+    res = oracle.osk(inp, order, count, eps)
+    q = inp.q.long().numpy()
+    k = inp.k.long().numpy()
+    off = Nkv - Nq
+    for h in range(Hq):
+        for I in range(wl.n_qblocks):
+            i = h * wl.n_qblocks + I
+            r0, r1 = I * bq, min((I + 1) * bq, Nq)
+            L = q[0, h, r0:r1] @ k[0, h // G].T
+            pos = off + np.arange(r0, r1)[:, None]
+            valid = np.arange(Nkv)[None, :] <= pos
+            m_run = np.full(r1 - r0, -np.inf)
+            for t in range(count[i].item()):
+                j = order[i, t].item()
+                c0, c1 = j * bk, min((j + 1) * bk, Nkv)
+                blk = np.where(valid[:, c0:c1], L[:, c0:c1], -np.inf)
+                m_loc = blk.max(1)
+                with np.errstate(invalid="ignore"):          # -inf - -inf on rows the mask leaves out
+                    vote = (m_loc == -np.inf) | (np.isfinite(m_run) & (m_loc - m_run < T))
+                skip = bool(vote.all())
+                assert res["skipped"][i, t].item() == int(skip), (h, I, t)
+                if not skip:
+                    m_run = np.maximum(m_run, m_loc)
+
+
 # ----------------------------------------------------------------- attention-mass recall of M_KAP
 
 def test_mass_recall_identity():
