@@ -388,6 +388,26 @@ def test_osk_eps0_equals_block_masked_sdpa(shape):
     assert torch.allclose(full_rows(res, wl), ref, atol=1e-12, rtol=0)
 
 
+@settings(max_examples=20, deadline=None, derandomize=True)
+@given(B=st.sampled_from([1, 2]), hq_g=st.sampled_from([(1, 1), (2, 1), (4, 2), (4, 4)]),
+       bq=st.sampled_from([32, 64, 128]), bk=st.sampled_from([32, 64, 128]), nq_units=st.integers(1, 20),
+       off_units=st.integers(0, 20), frac=st.sampled_from([0.2, 0.5, 1.0]), paged=st.booleans(),
+       wid=st.integers(0, 500))
+def test_osk_eps0_equals_block_masked_sdpa_random(B, hq_g, bq, bk, nq_units, off_units, frac, paged, wid):
+    """The same identity over random shapes: ragged blocks, queries after a
+    cache, GQA groups, batches, a paged cache, random block subsets."""
+    Hq, G = hq_g
+    Nq = 16 * nq_units
+    Nkv = Nq + 16 * off_units
+    wl = tiny(d=32, wid=wid, B=B, Hq=Hq, Hkv=Hq // G, Nq=Nq, Nkv=Nkv, bq=bq, bk=bk, paged=paged)
+    inp = synth.generate(wl)
+    order, count, allowed = _random_orders(wl, frac, wid)
+    res = oracle.osk(inp, order, count, 0.0)
+    assert res["skipped"].sum().item() == 0
+    ref = sdpa_reference(inp, allowed)
+    assert torch.allclose(full_rows(res, wl), ref, atol=1e-12, rtol=0)
+
+
 def test_full_budget_eps0_equals_dense():
     wl = tiny(Hq=4, Hkv=2, Nq=384, Nkv=384, bq=128, bk=128, structured=True, n_needle=1)
     inp = synth.generate(wl)
