@@ -638,6 +638,29 @@ def test_decode_kap_equals_prefill_kap_of_a_repeated_query(bk):
         assert torch.equal(dec["hrm"], ref["hrm"])
 
 
+@settings(max_examples=20, deadline=None, derandomize=True)
+@given(B=st.sampled_from([1, 2]), hq_g=st.sampled_from([(1, 1), (2, 1), (4, 2), (4, 4)]),
+       bk=st.sampled_from([32, 64, 128]), kv_units=st.integers(1, 60), budget=st.sampled_from([0.05, 0.2, 0.5, 1.0]),
+       seed=st.integers(0, 10_000))
+def test_decode_kap_equals_prefill_kap_random(B, hq_g, bk, kv_units, budget, seed):
+    """The same equivalence over random cache lengths (a ragged last block),
+    block sizes, GQA groups, batches and budgets."""
+    Hq, G = hq_g
+    Hkv, Nkv, d = Hq // G, 16 * kv_units, 32
+    g = torch.Generator().manual_seed(seed)
+    q = (torch.randn(B, Hq, d, generator=g) * 2).to(torch.bfloat16)
+    k = torch.randn(B, Hkv, Nkv, d, generator=g).to(torch.bfloat16)
+    dec = oracle.decode_kap(q, k, bk, 16, budget)
+    wl = tiny(B=B, Hq=Hq, Hkv=Hkv, Nq=16, Nkv=Nkv, d=d, bq=16, bk=bk)
+    qq = q[:, :, None, :].expand(B, Hq, 16, d).contiguous()
+    ref = oracle.kap(synth.Inputs(wl, qq, k.contiguous(), k.contiguous()), budget, want_scores=True)
+    assert torch.equal(dec["order"], ref["order"][:, : dec["order"].shape[1]])
+    assert torch.equal(dec["count"], ref["count"])
+    assert torch.equal(dec["hrm_count"], ref["hrm_count"])
+    assert torch.equal(dec["score"], ref["score"])
+    assert torch.equal(dec["hrm"], ref["hrm"])
+
+
 def test_decode_osk_eps0_is_dense_attention_of_the_row():
     """With eps = 0 nothing is skipped, and visiting every block in any order
     is softmax attention of the one query row over the whole cache
