@@ -45,6 +45,7 @@ def _shape(cosa, wl, paged, num_pages):
 DECODE_SHAPES = [
     dict(B=2, Hq=4, Hkv=2, Nq=2048, Nkv=2048, bk=128),
     dict(B=1, Hq=8, Hkv=2, Nq=1024, Nkv=3072, bk=64),
+    dict(B=1, Hq=4, Hkv=2, Nq=1040, Nkv=1040, bk=128),     # ragged cache: one pooled key in the last block
 ]
 
 
