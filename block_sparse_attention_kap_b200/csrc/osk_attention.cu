@@ -243,16 +243,36 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         if (!wait_or_abort(&sm->decided, ph, abort, p.status, DEV_TIMEOUT_PIPE)) break;
         const uint32_t dec = *reinterpret_cast<volatile uint32_t*>(&sm->decision);
         if (dec == kDecisionCompute) {
-          load(ks, &tm_v, order_at(t));
+          const int jv = order_at(t);
+          load(ks, &tm_v, jv);
           if (!wait_or_abort(&sm->p_ready, ph, abort, p.status, DEV_TIMEOUT_PIPE)) break;
           if (!wait_slot(ks)) break;
+          // A ragged last block: the V rows past the end of the cache are not
+          // keys (another head's rows, zero fill, or whatever a page's tail
+          // holds, NaN included).  Their P is 0, but 0 * NaN is NaN inside the
+          // MMA, so the 16-key steps past the end are not issued and the rows
+          // of the last issued step past the end are zeroed in shared memory
+          // (whole 128-byte rows: the swizzle permutes within a row).
+          const int valid = (jv >= 0 && jv < p.nkb) ? min(BK, p.Nkv - jv * BK) : BK;   // >= 1
+          const int ksteps = (valid + 15) >> 4;
+          if (valid < 16 * ksteps) {
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+            for (int c = 0; c < 2; ++c)
+              for (int r = valid; r < 16 * ksteps; ++r) {
+                uint4* dst = reinterpret_cast<uint4*>(slot(ks) + c * Cfg::kChunk + r * 128);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) dst[u] = z;
+              }
+            fence_proxy_async_smem();                          // visible to the tensor core's reads
+          }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
             // P of keys [16kk, 16kk+16): each column half packs its P at the
             // start of its own S range (TMEM columns half*BK/2 + ...)
-            mma_ts(tO, tS + (kk / (BK / 32)) * (BK / 2) + (kk % (BK / 32)) * 8,
-                   desc_sw128(slot_addr(ks) + kk * 2048, Cfg::kChunk, 1024), id_pv, (any_pv || kk > 0) ? 1u : 0u);
+            if (kk < ksteps)
+              mma_ts(tO, tS + (kk / (BK / 32)) * (BK / 2) + (kk % (BK / 32)) * 8,
+                     desc_sw128(slot_addr(ks) + kk * 2048, Cfg::kChunk, 1024), id_pv, (any_pv || kk > 0) ? 1u : 0u);
           any_pv = true;
           if (t + 2 < n) pend_k = t + 2;
         }

@@ -72,20 +72,28 @@ def flat(t):
     return t.reshape(-1, t.shape[-1]).cpu()
 
 
-def check_out(gpu_rows, ref_rows, extra_atol=None):
+def check_out(gpu_rows, ref_rows, extra_atol=None, literal=False):
     """Max error against the exact (fp64) oracle output, allowing half a
     bf16 ulp of the value; mean error against the oracle output rounded to
     bf16 (nearest even), the closest any bf16 output can be -- on outputs of
-    magnitude ~2 the rounding alone averages ~1.2e-3."""
+    magnitude ~2 the rounding alone averages ~1.2e-3.
+    literal=True applies the acceptance bar as written instead: max abs
+    error <= 1e-2 and mean abs error <= 1e-3, both against the exact oracle
+    output (used on the N(0,1) workloads, whose outputs stay below 4, where a
+    bf16 value can always be within 1e-2 of the exact one)."""
     g = gpu_rows.double().cpu()
     r = ref_rows.double().cpu()
     err = (g - r).abs()
-    tol = ATOL + RTOL * r.abs()
+    if literal:
+        assert r.abs().max().item() < 4.0, "an output of 4 or more cannot meet 1e-2 in bf16"
+        tol = torch.full_like(r, ATOL)
+    else:
+        tol = ATOL + RTOL * r.abs()
     if extra_atol is not None:
         tol = tol + extra_atol
     assert bool((err <= tol).all()), f"max abs err {err.max().item():.4g}"
-    mean_err = (g - oracle.round_bf16(r)).abs().mean().item()
-    assert mean_err <= MEAN_TOL, f"mean abs err (vs bf16-rounded oracle) {mean_err:.4g}"
+    mean_err = (g - (r if literal else oracle.round_bf16(r))).abs().mean().item()
+    assert mean_err <= MEAN_TOL, f"mean abs err (vs {'exact' if literal else 'bf16-rounded'} oracle) {mean_err:.4g}"
     return err.max().item()
 
 
@@ -190,11 +198,11 @@ def test_single_head_2k_normal(cosa):
     count = ref["count"].view(wl.B, wl.Hq, wl.n_qblocks).cuda()
     res = gpu_attend(m, dev, order, count, EPS)
     o = oracle.osk(inp, ref["order"], ref["count"], EPS)
-    check_skips_and_out(cosa, res, o, wl, ref["order"].shape[1])
+    check_skips_and_out(cosa, res, o, wl, ref["order"].shape[1], literal=True)
     # budget 100%, threshold 0 == dense attention
     full = m.plan(dev[0], dev[1], 1.0)
     res = gpu_attend(m, dev, full["order"], full["count"], 0.0)
-    check_out(gpu_rows(res["out"], wl), oracle.dense(inp)["out"])
+    check_out(gpu_rows(res["out"], wl), oracle.dense(inp)["out"], literal=True)
 
 
 def compare_plans(cosa, plan, ref, wl, budget, sel_idx=None):
@@ -224,11 +232,23 @@ def compare_plans(cosa, plan, ref, wl, budget, sel_idx=None):
         keys = sorted(range(n), key=lambda j: (-int(gh[i, j]), -float(gs[i, j]), j))
         assert go[i, :k].tolist() == keys[:k]
         assert bool((go[i, k:] == -1).all())
-        mism += sum(a != b for a, b in zip(go[i, :k].tolist(), ref["order"][i, :k].tolist()))
+        # a position where the two orders differ must hold a near-tie: the
+        # oracle's scores of the two blocks there within twice the score
+        # tolerance (HRM blocks score exactly 0, so an HRM near-tie counts)
+        for a, b in zip(go[i, :k].tolist(), ref["order"][i, :k].tolist()):
+            if a != b:
+                mism += 1
+                gap = abs(float(rs[i, a]) - float(rs[i, b]))
+                assert gap <= 2 * SCORE_TOL, f"row {i}: blocks {a} / {b} differ by {gap:.4g} in the oracle's score"
+    print(f"order positions that differ from the oracle's (all near-ties): {mism}")
     return mism
 
 
-def check_skips_and_out(cosa, res, o, wl, km, sel_idx=None):
+def check_skips_and_out(cosa, res, o, wl, km, sel_idx=None, eps=EPS, literal=False):
+    """Skip bits equal the oracle's except where its margin (pinned against
+    the definition in the oracle tests) is within MARGIN_TOL of 0, i.e. where
+    fp32 tensor-core logits may fall on the other side of the threshold;
+    outputs within tolerance, plus the derived allowance for each flip."""
     bits = cosa.unpack_skip_bits(flat(res["skip_bits"]), km)
     out = gpu_rows(res["out"], wl)
     if sel_idx is not None:
@@ -238,8 +258,14 @@ def check_skips_and_out(cosa, res, o, wl, km, sel_idx=None):
     assert bool((~diff | fragile).all()), "a robust skip decision differs"
     # a flipped decision moves a row by at most 2*max|v|*bk*eps
     flips = diff.sum(1).double()
-    extra = (2 * 6.0 * wl.bk * EPS * flips).view(-1, 1, 1)
-    return check_out(out, o["out"], extra_atol=extra), int(diff.sum())
+    vmax = 6.0
+    extra = (2 * vmax * wl.bk * eps * flips).view(-1, 1, 1)
+    n_flip = int(diff.sum())
+    print(f"skip decisions that differ from the oracle's (all within the margin): {n_flip} "
+          f"of {int(bits.numel())} entries; fragile visits {int(fragile.sum())}")
+    if literal and n_flip == 0:
+        extra = None
+    return check_out(out, o["out"], extra_atol=extra, literal=literal), n_flip
 
 
 def test_order_invariance_gpu(cosa):
@@ -308,12 +334,47 @@ def _samples(wl, n, seed):
     return sorted(picks)
 
 
-@pytest.mark.parametrize("name,budget", [("gqa_32k", 0.1), ("gqa_128k", 0.1), ("chunked_128k_paged", 0.1),
-                                         ("sweep_64k_b2", 0.05)])
-def test_full_size_sampled(cosa, name, budget):
+_FULL = {}
+
+
+def _full_inputs(cosa, name, grid):
+    """The workload's inputs on host and device, kept for the next case of
+    the same workload (only one workload is held at a time)."""
+    key = (name, grid)
+    if key not in _FULL:
+        _FULL.clear()
+        torch.cuda.empty_cache()
+        inp = synth.generate(synth.WORKLOADS[name], grid=grid)
+        _FULL[key] = (inp, to_gpu(inp))
+    return _FULL[key]
+
+
+# every workload and budget of the benchmark plan, at its own full size: the
+# 2K single head at 25%, the 32K layer at 10%, the 128K layer at 10% and 5%,
+# the 4096-query chunk after a 128K paged cache at 10%, and the B=2 x 64K
+# sweep at 100% (threshold 0: must equal dense attention), 50, 20, 10, 5, 2%
+FULL_CASES = [("single_head_2k", 0.25, EPS), ("gqa_32k", 0.1, EPS), ("gqa_128k", 0.1, EPS), ("gqa_128k", 0.05, EPS),
+              ("chunked_128k_paged", 0.1, EPS), ("sweep_64k_b2", 1.0, 0.0), ("sweep_64k_b2", 0.5, EPS),
+              ("sweep_64k_b2", 0.2, EPS), ("sweep_64k_b2", 0.1, EPS), ("sweep_64k_b2", 0.05, EPS),
+              ("sweep_64k_b2", 0.02, EPS)]
+
+
+@pytest.mark.parametrize("name,budget,eps", FULL_CASES)
+def test_full_size_sampled(cosa, name, budget, eps):
+    """N(0,1)-based inputs at full size, in the launch configuration the
+    benchmark times (one plan and one attend over the whole problem): on 12
+    sampled (b, head, Q-block) rows the plan agrees with the oracle's (scores
+    within SCORE_TOL, orders equal up to near-ties), skip bits equal except
+    where the margin is within MARGIN_TOL, and outputs meet the acceptance
+    bar as written (max abs <= 1e-2, mean abs <= 1e-3 against the exact
+    oracle).  At budget 100% with threshold 0 the output is also compared
+    with dense causal attention."""
     wl = synth.WORKLOADS[name]
-    inp = synth.generate(wl)
-    m, dev, plan = gpu_plan(cosa, inp, budget)
+    inp, dev = _full_inputs(cosa, name, False)
+    m = cosa.CoSA(cosa.shape_of_workload(wl))
+    plan = m.plan(dev[0], dev[1], budget, page_table=dev[3], scores=True)
+    torch.cuda.synchronize()
+    assert m.device_status() == 0
     sel = _samples(wl, 12, 3)
     idx = [(b * wl.Hq + h) * wl.n_qblocks + I for b, h, I in sel]
     km = plan["order"].shape[-1]
@@ -324,9 +385,53 @@ def test_full_size_sampled(cosa, name, budget):
     count = plan["count"].clone().view(-1)
     order[idx] = ref["order"].cuda()
     count[idx] = ref["count"].cuda()
-    res = gpu_attend(m, dev, order.view_as(plan["order"]), count.view_as(plan["count"]), EPS)
-    o = oracle.osk(inp, ref["order"], ref["count"], EPS, sel=sel)
-    check_skips_and_out(cosa, res, o, wl, km, sel_idx=idx)
+    res = gpu_attend(m, dev, order.view_as(plan["order"]), count.view_as(plan["count"]), eps)
+    o = oracle.osk(inp, ref["order"], ref["count"], eps, sel=sel)
+    check_skips_and_out(cosa, res, o, wl, km, sel_idx=idx, eps=eps, literal=True)
+    if budget == 1.0 and eps == 0.0:
+        assert int(cosa.unpack_skip_bits(flat(res["skip_bits"]), km).sum()) == 0
+        dense = oracle.dense(inp, sel=sel)
+        check_out(gpu_rows(res["out"], wl)[idx], dense["out"], literal=True)
+
+
+GRID_FULL_CASES = [("single_head_2k", 0.25), ("gqa_32k", 0.1), ("gqa_128k", 0.1), ("gqa_128k", 0.05),
+                   ("chunked_128k_paged", 0.1), ("sweep_64k_b2", 1.0), ("sweep_64k_b2", 0.5),
+                   ("sweep_64k_b2", 0.2), ("sweep_64k_b2", 0.1), ("sweep_64k_b2", 0.05), ("sweep_64k_b2", 0.02)]
+
+
+@pytest.mark.parametrize("name,budget", GRID_FULL_CASES)
+def test_full_size_grid_bit_exact(cosa, name, budget):
+    """Each workload at its own full shape (GQA 32/8 at 32K, 128K and B=2 x
+    64K, the paged 128K chunk, the 2K single head) on structured integer-grid
+    inputs, where every pooled value and logit is exact: on sampled (b, head,
+    Q-block) rows the GPU's order, count, HRM count, block scores and HRM
+    flags equal the oracle's bit for bit, and so do the in-kernel skip bits
+    of the attend over the GPU's own plan (eps 1e-4; at budget 100% also
+    with eps 0, where nothing may be skipped)."""
+    wl = synth.WORKLOADS[name]
+    inp, dev = _full_inputs(cosa, name, True)
+    m = cosa.CoSA(cosa.shape_of_workload(wl))
+    plan = m.plan(dev[0], dev[1], budget, page_table=dev[3], scores=True)
+    torch.cuda.synchronize()
+    assert m.device_status() == 0
+    n_rows = wl.B * wl.Hq * wl.n_qblocks
+    sel = _samples(wl, 12, 5) if n_rows > 64 else None
+    idx = [(b * wl.Hq + h) * wl.n_qblocks + I for b, h, I in sel] if sel else list(range(n_rows))
+    km = plan["order"].shape[-1]
+    ref = oracle.kap(inp, budget, sel=sel, kmax_=km, want_scores=True)
+    assert torch.equal(flat(plan["count"]).view(-1)[idx], ref["count"])
+    assert torch.equal(flat(plan["order"])[idx], ref["order"])
+    assert torch.equal(flat(plan["hrm_count"]).view(-1)[idx], ref["hrm_count"])
+    assert torch.equal(flat(plan["block_score"])[idx], ref["score"])
+    assert torch.equal(flat(plan["hrm"])[idx], ref["hrm"])
+    for eps in ((EPS, 0.0) if budget == 1.0 else (EPS,)):
+        res = gpu_attend(m, dev, plan["order"], plan["count"], eps)
+        o = oracle.osk(inp, ref["order"], ref["count"], eps, sel=sel)
+        bits = cosa.unpack_skip_bits(flat(res["skip_bits"]), km)[idx]
+        assert torch.equal(bits, o["skipped"])
+        if eps == 0.0:
+            assert int(bits.sum()) == 0
+        check_out(gpu_rows(res["out"], wl)[idx], o["out"])
 
 
 def test_mass_recall_matches_oracle(cosa):

@@ -135,6 +135,14 @@ def test_osk_hand_example():
         exp3 = dense3 if f["out3"] == "dense" else named[f["out3"]]
         assert o[1, 0, 0].item() == pytest.approx(exp2, abs=1e-12)
         assert o[1, 1, 0].item() == pytest.approx(exp3, abs=1e-12)
+        # skip margins: mdiff (by hand) minus T, +inf where a row had no running max
+        T = float(np.float32(math.log(eps))) if eps > 0 else -math.inf
+        want = [math.inf if x == "inf" else float(x) - T for x in f["mdiff"].split(",")]
+        mg = res["margin"]
+        assert mg[0, 0].item() == math.inf and math.isnan(mg[0, 1].item())
+        assert mg[1].tolist() == want
+        if eps > 0:
+            assert [int(x < 0) for x in want] == res["skipped"][1].tolist()
 
 
 def test_skip_threshold_value():
@@ -461,6 +469,7 @@ def test_skip_decisions_bruteforce_grid():
     plan = oracle.kap(inp, 1.0)
     eps = 1e-3
     T = math.log(eps) * math.sqrt(wl.d)
+    T32 = np.float32(T)
     res = oracle.osk(inp, plan["order"], plan["count"], eps)
     q = inp.q.long().numpy()
     k = inp.k.long().numpy()
@@ -479,9 +488,25 @@ def test_skip_decisions_bruteforce_grid():
                 vote = (m_loc == -np.inf) | (np.isfinite(m_run) & (m_loc - m_run < T))
                 skip = bool(vote.all())
                 assert res["skipped"][i, t].item() == int(skip)
+                assert res["margin"][i, t].item() == _margin_by_definition(m_loc, m_run, T32)
                 if not skip:
                     m_run = np.maximum(m_run, m_loc)
     assert res["skipped"].sum().item() > 0          # decisions of both kinds were checked
+
+
+def _margin_by_definition(m_loc, m_run, T32):
+    """The skip margin of one visit from its definition: over the rows whose
+    m_loc is finite, the largest fp32(m_loc - m_run) - T (fp32 subtraction,
+    then the difference to T in fp64); +inf if such a row has no running max
+    yet or T = -inf (eps = 0); -inf if no row sees a key of the block.  The
+    block is skipped iff this is negative (every row then votes skip)."""
+    seen = np.isfinite(m_loc)
+    if not seen.any():
+        return -math.inf
+    if not np.isfinite(T32) or not np.isfinite(m_run[seen]).all():
+        return math.inf
+    diff = np.float32(m_loc[seen]).astype(np.float32) - np.float32(m_run[seen]).astype(np.float32)
+    return float(diff.astype(np.float32).max()) - float(T32)
 
 
 @settings(max_examples=25, deadline=None, derandomize=True)
@@ -499,6 +524,7 @@ def test_skip_decisions_bruteforce_random(hq_g, bq, bk, nq_units, off_units, fra
     inp = synth.generate(wl, grid=True)
     order, count, _ = _random_orders(wl, frac, wid)
     T = math.log(eps) * math.sqrt(wl.d)
+    T32 = np.float32(T)
     res = oracle.osk(inp, order, count, eps)
     q = inp.q.long().numpy()
     k = inp.k.long().numpy()
@@ -520,7 +546,87 @@ def test_skip_decisions_bruteforce_random(hq_g, bq, bk, nq_units, off_units, fra
                     vote = (m_loc == -np.inf) | (np.isfinite(m_run) & (m_loc - m_run < T))
                 skip = bool(vote.all())
                 assert res["skipped"][i, t].item() == int(skip), (h, I, t)
+                assert res["margin"][i, t].item() == _margin_by_definition(m_loc, m_run, T32), (h, I, t)
                 if not skip:
+                    m_run = np.maximum(m_run, m_loc)
+
+
+def test_skip_margin_rounds_the_difference_to_fp32():
+    """The margin takes m_loc - m_run in fp32, as the skip test does (worked
+    by hand): one head, d = 1, blocks of one token, query 1 = 1024 visits key
+    0 = 1024 (logit 2^20, computed first) and then key 1 = (1 + 2^-7) / 1024
+    (logit 1 + 2^-7).  The exact difference -1048574.9921875 lies between the
+    fp32 neighbours -1048575 and -1048574.9375 (spacing 2^-4 below 2^20) and
+    rounds to -1048575, so the margin is -1048575 - T, not the exact
+    difference minus T."""
+    wl = tiny(Hq=1, Nq=2, Nkv=2, d=1, bq=1, bk=1, stride=1)
+    t = lambda x: torch.tensor(x, dtype=torch.float64).view(1, 1, 2, 1)
+    inp = inputs_from(wl, t([1.0, 1024.0]), t([1024.0, (1.0 + 2.0 ** -7) / 1024.0]), t([1.0, -1.0]))
+    assert inp.k[0, 0, 1, 0].double().item() == (1.0 + 2.0 ** -7) / 1024.0      # exact in bf16
+    order = torch.tensor([[0, -1], [0, 1]], dtype=torch.int32)
+    count = torch.tensor([1, 2], dtype=torch.int32)
+    eps = 1e-4
+    T32 = np.float32(math.log(eps))
+    res = oracle.osk(inp, order, count, eps)
+    assert res["margin"][1, 0].item() == math.inf
+    assert res["margin"][1, 1].item() == -1048575.0 - float(T32)
+    assert res["margin"][1, 1].item() != -1048574.9921875 - float(T32)
+    assert res["skipped"][1].tolist() == [0, 1]
+    assert res["out"][1, 0, 0].item() == 1.0          # the skipped key adds nothing
+
+
+@settings(max_examples=20, deadline=None, derandomize=True)
+@given(hq_g=st.sampled_from([(1, 1), (2, 1), (4, 2)]), bq=st.sampled_from([32, 64]), bk=st.sampled_from([32, 64]),
+       nq_units=st.integers(1, 12), off_units=st.integers(0, 12), frac=st.sampled_from([0.3, 0.7, 1.0]),
+       eps=st.sampled_from([0.0, 1e-4, 1e-2, 0.3]), wid=st.integers(0, 500))
+def test_skip_margin_bruteforce_normal(hq_g, bq, bk, nq_units, off_units, frac, eps, wid):
+    """The skip margin on real-valued (N(0,1) plus structure) inputs, which
+    the GPU parity tests use to tell fragile skip decisions from robust ones:
+    recomputed from its definition with numpy fp64 logits rounded to fp32
+    (the products are summed in another order than the oracle's, so the
+    comparison allows 1e-3 raw-logit units), decisions exact wherever the
+    margin is farther than that from 0, and, from the oracle alone, a
+    negative margin exactly on the skipped visits (+inf everywhere at eps 0)."""
+    Hq, G = hq_g
+    Nq = 16 * nq_units
+    Nkv = Nq + 16 * off_units
+    wl = tiny(d=32, wid=wid, Hq=Hq, Hkv=Hq // G, Nq=Nq, Nkv=Nkv, bq=bq, bk=bk, structured=True, n_needle=1)
+    inp = synth.generate(wl)
+    order, count, _ = _random_orders(wl, frac, wid)
+    T = oracle.skip_threshold(eps, wl.d)
+    T32 = np.float32(T)
+    res = oracle.osk(inp, order, count, eps)
+    q = inp.q.double().numpy()
+    k = inp.k.double().numpy()
+    off = Nkv - Nq
+    for h in range(Hq):
+        for I in range(wl.n_qblocks):
+            i = h * wl.n_qblocks + I
+            n = count[i].item()
+            mg = res["margin"][i, :n]
+            sk = res["skipped"][i, :n].bool()
+            if eps == 0.0:
+                assert bool(torch.isinf(mg).all() & (mg > 0).all()) and not sk.any()
+            else:
+                assert torch.equal(sk, mg < 0)
+            r0, r1 = I * bq, min((I + 1) * bq, Nq)
+            L = (q[0, h, r0:r1] @ k[0, h // G].T).astype(np.float32)
+            pos = off + np.arange(r0, r1)[:, None]
+            valid = np.arange(Nkv)[None, :] <= pos
+            m_run = np.full(r1 - r0, -np.inf, dtype=np.float32)
+            for t in range(n):
+                j = order[i, t].item()
+                c0, c1 = j * bk, min((j + 1) * bk, Nkv)
+                m_loc = np.where(valid[:, c0:c1], L[:, c0:c1], -np.inf).max(1).astype(np.float32)
+                want = _margin_by_definition(m_loc, m_run, T32)
+                got = mg[t].item()
+                if math.isinf(want):
+                    assert got == want, (h, I, t)
+                else:
+                    assert abs(got - want) <= 1e-3, (h, I, t, got, want)
+                if abs(want) > 1e-3:
+                    assert bool(sk[t]) == (want < 0)
+                if not sk[t]:
                     m_run = np.maximum(m_run, m_loc)
 
 
