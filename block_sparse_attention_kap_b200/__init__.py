@@ -62,6 +62,7 @@ _lib.cosa_decode_plan.argtypes = [_S, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int
                                   _P, _P, _P, _P, _P, _P]
 _lib.cosa_plan_static.argtypes = [_S, _P, _P, _P, ctypes.c_double, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P]
 _lib.cosa_attend.argtypes = [_S, _P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_double, _P, _P, _P, _P, _P]
+_lib.cosa_test_attend_wait_timeout.argtypes = [_S, _P, _P, _P, _P, _P, _P, ctypes.c_int, _P, _P, ctypes.c_uint64, _P]
 _lib.cosa_skip_threshold.argtypes = [ctypes.c_double, ctypes.c_int]
 _lib.cosa_skip_threshold.restype = ctypes.c_float
 _lib.cosa_status_string.argtypes = [ctypes.c_int]
@@ -69,7 +70,9 @@ _lib.cosa_status_string.restype = ctypes.c_char_p
 
 EXPORTS = ("cosa_num_qblocks", "cosa_num_kblocks", "cosa_kmax", "cosa_plan_workspace_bytes", "cosa_plan",
            "cosa_dense_order", "cosa_attend", "cosa_skip_threshold", "cosa_status_string", "cosa_version",
-           "cosa_plan_static", "cosa_plan_chunk", "cosa_block_union", "cosa_decode_plan")
+           "cosa_plan_static", "cosa_plan_chunk", "cosa_block_union", "cosa_decode_plan",
+           "cosa_test_attend_wait_timeout")
+DEV_TIMEOUT_TMA, DEV_TIMEOUT_MMA, DEV_TIMEOUT_PIPE = 0x100, 0x200, 0x300
 STATIC_SCRATCH_BYTES = 64 << 20
 
 
@@ -217,6 +220,20 @@ def cosa_attend(shape: cosa_shape, q, k, v, page_table, order, count, kmax: int,
                             _ptr(out, "out", torch.bfloat16), _ptr(lse, "lse", torch.float32),
                             _ptr(skip_bits, "skip_bits", torch.int32), _ptr(dev_status, "dev_status", torch.int32),
                             _stream(stream)), "cosa_attend")
+
+
+def cosa_test_attend_wait_timeout(shape: cosa_shape, q, k, v, page_table, order, count, kmax: int, out,
+                                  dev_status, wait_limit_ns: int, stream=None) -> None:
+    """Failure-detection test hook: cosa_attend's kernel with one wait per
+    CTA that nothing completes, so every bounded wait gives up after
+    wait_limit_ns and the kernel reports DEV_TIMEOUT_PIPE in dev_status."""
+    _check(_lib.cosa_test_attend_wait_timeout(ctypes.byref(shape), _ptr(q, "q", torch.bfloat16),
+                                              _ptr(k, "k", torch.bfloat16), _ptr(v, "v", torch.bfloat16),
+                                              _ptr(page_table, "page_table", torch.int32),
+                                              _ptr(order, "order", torch.int32), _ptr(count, "count", torch.int32),
+                                              kmax, _ptr(out, "out", torch.bfloat16),
+                                              _ptr(dev_status, "dev_status", torch.int32), wait_limit_ns,
+                                              _stream(stream)), "cosa_test_attend_wait_timeout")
 
 
 # ----------------------------------------------------------------- convenience (allocation via torch)

@@ -354,10 +354,14 @@ cosa_status cosa_block_union(const cosa_shape* shape, const int32_t* order, cons
   return launch_status(launch_block_union(p, stream));
 }
 
-cosa_status cosa_attend(const cosa_shape* shape, const void* q, const void* k, const void* v,
+}  // extern "C"
+
+namespace {
+
+cosa_status attend_impl(const cosa_shape* shape, const void* q, const void* k, const void* v,
                         const int32_t* page_table, const int32_t* order, const int32_t* count, int kmax,
                         double skip_eps, void* out, float* lse, uint32_t* skip_bits, uint32_t* dev_status,
-                        cudaStream_t stream) {
+                        uint64_t wait_limit_ns, int stall_test, cudaStream_t stream) {
   cosa_status st = check_shape(shape);
   if (st != COSA_OK) return st;
   if (!(skip_eps >= 0.0) || skip_eps >= 1.0) return COSA_EINVAL;
@@ -381,7 +385,30 @@ cosa_status cosa_attend(const cosa_shape* shape, const void* q, const void* k, c
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)s.d));
   p.out = static_cast<uint16_t*>(out); p.lse = lse; p.skip_bits = skip_bits; p.skip_words = cdiv(kmax, 32);
   p.status = dev_status;
+  p.wait_limit_ns = wait_limit_ns;
+  p.stall_test = stall_test;
   return launch_status(launch_osk(tm_q, tm_k, tm_v, p, s.bk, stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+cosa_status cosa_attend(const cosa_shape* shape, const void* q, const void* k, const void* v,
+                        const int32_t* page_table, const int32_t* order, const int32_t* count, int kmax,
+                        double skip_eps, void* out, float* lse, uint32_t* skip_bits, uint32_t* dev_status,
+                        cudaStream_t stream) {
+  return attend_impl(shape, q, k, v, page_table, order, count, kmax, skip_eps, out, lse, skip_bits, dev_status,
+                     1000000000ull, 0, stream);
+}
+
+cosa_status cosa_test_attend_wait_timeout(const cosa_shape* shape, const void* q, const void* k, const void* v,
+                                          const int32_t* page_table, const int32_t* order, const int32_t* count,
+                                          int kmax, void* out, uint32_t* dev_status, uint64_t wait_limit_ns,
+                                          cudaStream_t stream) {
+  if (!dev_status || wait_limit_ns < 1000ull || wait_limit_ns > 1000000000ull) return COSA_EINVAL;
+  return attend_impl(shape, q, k, v, page_table, order, count, kmax, 0.0, out, nullptr, nullptr, dev_status,
+                     wait_limit_ns, 1, stream);
 }
 
 const char* cosa_status_string(cosa_status status) {

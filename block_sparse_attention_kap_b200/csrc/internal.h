@@ -91,6 +91,8 @@ struct OskParams {
   uint32_t* skip_bits;          // optional [B, Hq, nQB, skip_words]
   int skip_words;
   uint32_t* status;
+  uint64_t wait_limit_ns;       // limit of every pipeline wait (1 s; shorter only in the test hook)
+  int stall_test;               // 0; 1 only in the wait-timeout test hook
 };
 cudaError_t launch_osk(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                        const OskParams& p, int bk, cudaStream_t st);

@@ -52,6 +52,7 @@ constexpr int kOrderCap = 1024;                            // order entries stag
 
 struct __align__(8) OskSmem {
   uint64_t q_full, full[2], s_full, decided, p_ready, o_final;
+  uint64_t never;               // nothing ever arrives here (the wait-timeout test hook waits on it)
   uint32_t decision;
   uint32_t tmem_base;
   uint32_t abort;               // set once any wait of this CTA gave up
@@ -173,6 +174,7 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     mbar_init(&sm->decided, 1);
     mbar_init(&sm->p_ready, kSoftmaxThreads);
     mbar_init(&sm->o_final, 1);
+    mbar_init(&sm->never, 1);
     sm->abort = 0;
     fence_mbar_init();
   }
@@ -209,7 +211,7 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         tma_load_2d(slot(sl) + Cfg::kChunk, tm, &sm->full[sl], 64, y);
       };
       auto wait_slot = [&](int sl) {
-        const bool r = wait_or_abort(&sm->full[sl], (fph >> sl) & 1u, abort, p.status, DEV_TIMEOUT_TMA);
+        const bool r = wait_or_abort(&sm->full[sl], (fph >> sl) & 1u, abort, p.status, DEV_TIMEOUT_TMA, p.wait_limit_ns);
         if (r) {
           fph ^= 1u << sl;
           busy &= ~(1u << sl);
@@ -229,23 +231,26 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       load(0, &tm_k, order_at(0));
       if (n > 1) load(1, &tm_k, order_at(1));
       bool any_pv = false;
-      const bool q_seen = wait_or_abort(&sm->q_full, 0, abort, p.status, DEV_TIMEOUT_TMA);
+      const bool q_seen = wait_or_abort(&sm->q_full, 0, abort, p.status, DEV_TIMEOUT_TMA, p.wait_limit_ns);
       bool ok = q_seen && wait_slot(0);
+      // failure-detection test hook: a wait that cannot complete, so the
+      // bounded wait gives up and every thread takes the abort path
+      if (ok && p.stall_test) ok = wait_or_abort(&sm->never, 0, abort, p.status, DEV_TIMEOUT_PIPE, p.wait_limit_ns);
       if (ok) { tc_fence_after(); issue_qk(0); }
       int ks = 0;            // slot holding K of visit t
       int pend_k = -1;       // K load deferred until the PV reading its slot has completed
       for (int t = 0; ok && t < n; ++t) {
         const uint32_t ph = t & 1;
         const int ns = ks ^ 1;
-        if (!wait_or_abort(&sm->s_full, ph, abort, p.status, DEV_TIMEOUT_MMA)) break;
+        if (!wait_or_abort(&sm->s_full, ph, abort, p.status, DEV_TIMEOUT_MMA, p.wait_limit_ns)) break;
         // QK_t and every earlier MMA are complete
         if (pend_k >= 0) { load(ns, &tm_k, order_at(pend_k)); pend_k = -1; }
-        if (!wait_or_abort(&sm->decided, ph, abort, p.status, DEV_TIMEOUT_PIPE)) break;
+        if (!wait_or_abort(&sm->decided, ph, abort, p.status, DEV_TIMEOUT_PIPE, p.wait_limit_ns)) break;
         const uint32_t dec = *reinterpret_cast<volatile uint32_t*>(&sm->decision);
         if (dec == kDecisionCompute) {
           const int jv = order_at(t);
           load(ks, &tm_v, jv);
-          if (!wait_or_abort(&sm->p_ready, ph, abort, p.status, DEV_TIMEOUT_PIPE)) break;
+          if (!wait_or_abort(&sm->p_ready, ph, abort, p.status, DEV_TIMEOUT_PIPE, p.wait_limit_ns)) break;
           if (!wait_slot(ks)) break;
           // A ragged last block: the V rows past the end of the cache are not
           // keys (another head's rows, zero fill, or whatever a page's tail
@@ -318,7 +323,7 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       const int j = order_at(t);
       const bool j_ok = j >= 0 && j < p.nkb;
       // after a failure every thread still runs the same barriers, without waiting
-      const bool got = wait_or_abort(&sm->s_full, t & 1, abort, p.status, DEV_TIMEOUT_MMA);
+      const bool got = wait_or_abort(&sm->s_full, t & 1, abort, p.status, DEV_TIMEOUT_MMA, p.wait_limit_ns);
       tc_fence_after();
       const int lim = min(qpos - j * BK, p.Nkv - 1 - j * BK);   // last visible column
       // pass 1: max over this half's visible columns (one 64-column TMEM load
@@ -431,7 +436,7 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     // ------------------------------------------------------------ epilogue
     bool have_o = any_pv;
     if (n > 0) {
-      if (!wait_or_abort(&sm->o_final, 0, abort, p.status, DEV_TIMEOUT_MMA)) have_o = false;
+      if (!wait_or_abort(&sm->o_final, 0, abort, p.status, DEV_TIMEOUT_MMA, p.wait_limit_ns)) have_o = false;
       tc_fence_after();
     }
     sm->lx[half][r] = l;

@@ -81,9 +81,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
 // up (*abort set): after a failure every thread still runs through the same
 // barrier sequence, just without waiting, so no named barrier can hang.
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile uint32_t* abort,
-                                              uint32_t* status, uint32_t code) {
+                                              uint32_t* status, uint32_t code,
+                                              uint64_t limit_ns = 1000000000ull) {
   if (*abort) return false;
-  if (mbar_wait(bar, parity)) return true;
+  if (mbar_wait(bar, parity, limit_ns)) return true;
   *abort = 1u;
   report(status, code);
   return false;

@@ -215,6 +215,33 @@ COSA_API cosa_status cosa_attend(const cosa_shape* shape, const void* q, const v
                         double skip_eps, void* out, float* lse, uint32_t* skip_bits, uint32_t* dev_status,
                         cudaStream_t stream);
 
+/* Failure-detection test hook (no counterpart in the papers): runs
+ * cosa_attend's kernel with skip_eps = 0 on the given arguments, except that
+ * in every CTA the issuing thread, before the first QK^T, waits on a barrier
+ * that nothing ever arrives at.  That wait, like every other wait of the
+ * kernel, gives up after wait_limit_ns nanoseconds of %globaltimer; the
+ * kernel then records a timeout code in *dev_status (COSA_DEV_TIMEOUT_PIPE
+ * from that wait, or COSA_DEV_TIMEOUT_MMA from the softmax threads' wait for
+ * the QK^T that never comes, whichever gives up first), every thread
+ * runs through the rest of its barriers without waiting, the issuing thread
+ * waits (again bounded) for the copies it started, TMEM is released and the
+ * CTA exits; CTAs that start after the status is set exit at once.  The
+ * call returns COSA_OK; the CTAs that ran write zeros to their rows of
+ * `out`, the others leave them as they were; the context stays usable: a test calls it to check that a wait that runs out
+ * ends in an error status rather than a hang or a fault.  Not for use in
+ * production.
+ *  dev_status     required; should be 0 before the call.
+ *  wait_limit_ns  in [1e3, 1e9].
+ * Returns COSA_EINVAL for a null dev_status or a limit out of range, and
+ * otherwise what cosa_attend returns for the same arguments. */
+#define COSA_DEV_TIMEOUT_TMA 0x100u    /* device status: a TMA transaction never completed */
+#define COSA_DEV_TIMEOUT_MMA 0x200u    /* device status: a tensor-core commit never arrived */
+#define COSA_DEV_TIMEOUT_PIPE 0x300u   /* device status: a producer/consumer hand-off never arrived */
+COSA_API cosa_status cosa_test_attend_wait_timeout(const cosa_shape* shape, const void* q, const void* k,
+                                                   const void* v, const int32_t* page_table, const int32_t* order,
+                                                   const int32_t* count, int kmax, void* out, uint32_t* dev_status,
+                                                   uint64_t wait_limit_ns, cudaStream_t stream);
+
 /* cosa_plan without a workspace argument, for callers that cannot obtain
  * device memory of their own (for example a serving engine that reserves the
  * whole GPU at start-up and only hands kernels the tensors it owns, or a

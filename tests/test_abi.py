@@ -172,6 +172,21 @@ def test_attend_argument_errors_return_before_launch(cosa):
     assert call(shape=cosa.make_shape(1, 4, 2, 0, 512, 128, 128, 64, 16), q=None) == 0
 
 
+def test_wait_timeout_hook_argument_errors_return_before_launch(cosa):
+    lib = cosa._lib
+    s = cosa.make_shape(1, 4, 2, 256, 512, 128, 128, 64, 16)
+    P = 1 << 20
+
+    def call(status=P, limit=10 ** 6):
+        return lib.cosa_test_attend_wait_timeout(ctypes.byref(s), P, P, P, None, P, P, 8, P, status, limit, None)
+    assert call(status=None) == 1
+    assert call(limit=10) == 1
+    assert call(limit=2 * 10 ** 9) == 1
+    # the same validation as cosa_attend before any launch: a misaligned output
+    assert lib.cosa_test_attend_wait_timeout(ctypes.byref(s), P, P, P, None, P, P, 8, P + 8, P, 10 ** 6,
+                                             None) == 2
+
+
 def test_status_strings(cosa):
     for code in range(7):
         assert cosa.cosa_status_string(code).startswith("COSA_")

@@ -194,3 +194,49 @@ def test_nan_in_ragged_page_tail(cosa, bk, Nkv, eps):
     km = ref_order.shape[1]
     assert torch.equal(cosa.unpack_skip_bits(flat(res["skip_bits"]), km), o["skipped"])
     check_out(gpu_rows(res["out"], wl), o["out"])
+
+
+def test_bounded_wait_gives_up_and_reports(cosa):
+    """Failure detection on the GPU without a fault: the test hook makes one
+    wait per CTA of the attention kernel wait on a barrier nothing arrives
+    at.  Every wait of the kernel is bounded (here by 2 ms), so the kernel
+    must end by itself with a timeout code in the status word; CTAs that
+    ran write zero rows, CTAs that start after the report exit at once and
+    leave their rows untouched, and the context stays usable: the next
+    normal call on the same buffers is correct.  512 CTAs, more than the
+    GPU holds at once, so both kinds of CTA occur."""
+    import time
+    wl = tiny(Hq=8, Hkv=2, Nq=8192, Nkv=8192, bq=128, bk=128, structured=True, n_needle=4)
+    inp = synth.generate(wl, grid=True)
+    m = cosa.CoSA(cosa.shape_of_workload(wl))
+    q, k, v = inp.q.cuda(), inp.k.cuda(), inp.v.cuda()
+    plan = m.plan(q, k, 1.0)
+    km = plan["order"].shape[-1]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.full((wl.B, wl.Hq, wl.Nq, wl.d), 7.0, dtype=torch.bfloat16, device="cuda")
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    cosa.cosa_test_attend_wait_timeout(m.shape, q, k, v, None, plan["order"], plan["count"], km, out, status,
+                                       2_000_000)
+    torch.cuda.synchronize()
+    elapsed = time.perf_counter() - t0
+    code = int(status.item())
+    assert code in (cosa.DEV_TIMEOUT_PIPE, cosa.DEV_TIMEOUT_MMA), hex(code)
+    assert elapsed < 5.0
+    blocks = out.float().view(wl.B * wl.Hq * wl.n_qblocks, wl.bq * wl.d)
+    zero = (blocks == 0).all(1)
+    kept = (blocks == 7).all(1)
+    assert bool((zero | kept).all())
+    assert int(zero.sum()) > 0 and int(kept.sum()) > 0
+    # the same context and buffers, a normal call: correct on sampled rows
+    m.status.zero_()
+    res = m.attend(q, k, v, plan["order"], plan["count"], EPS, out=out, skip_bits=True)
+    torch.cuda.synchronize()
+    assert m.device_status() == 0
+    sel = [(0, 0, 63), (0, 3, 17), (0, 7, 0), (0, 5, 40)]
+    idx = [(b * wl.Hq + h) * wl.n_qblocks + I for b, h, I in sel]
+    ref = oracle.kap(inp, 1.0, sel=sel, kmax_=km)
+    assert torch.equal(flat(plan["order"])[idx], ref["order"])
+    o = oracle.osk(inp, ref["order"], ref["count"], EPS, sel=sel)
+    assert torch.equal(cosa.unpack_skip_bits(flat(res["skip_bits"]), km)[idx], o["skipped"])
+    check_out(gpu_rows(res["out"], wl)[idx], o["out"])
