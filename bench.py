@@ -346,6 +346,17 @@ def run_chunked(args, wl, budget, eps):
                                                            None, None, m.status, stream))
     attend_union_eps_ms = timed(lambda: cosa.cosa_attend(shape, q, k, v, pt, u_order, u_count, u_km, eps, out_u,
                                                          None, None, m.status, stream))
+    # the same union executed by the group kernel (one order per kv-head
+    # group, K/V tiles shared by two heads); its rows are the union's rows of
+    # the group's first head
+    G = wl.Hq // wl.Hkv
+    g_order = u_order.view(wl.B, wl.Hkv, G, m.nqb, u_km)[:, :, 0].contiguous()
+    g_count = u_count.view(wl.B, wl.Hkv, G, m.nqb)[:, :, 0].contiguous()
+    out_g = torch.empty_like(out)
+    group_dense_ms = timed(lambda: cosa.cosa_attend_group(shape, q, k, v, pt, g_order, g_count, u_km, 0.0, out_g,
+                                                           None, None, m.status, stream))
+    group_eps_ms = timed(lambda: cosa.cosa_attend_group(shape, q, k, v, pt, g_order, g_count, u_km, eps, out_g,
+                                                         None, None, m.status, stream))
     torch.cuda.synchronize()
     assert m.device_status() == 0
     assert torch.equal(order, full_order), "cached pooled keys changed the plan"
@@ -368,7 +379,8 @@ def run_chunked(args, wl, budget, eps):
         "kap_blocks": kap_blocks, "err_kap_vs_dense": err(kap_out),
         "union": {"union_ms": union_ms, "blocks": union_blocks, "attend_eps0_ms": attend_union_dense_ms,
                   "attend_eps_ms": attend_union_eps_ms,
-                  "step_eps0_ms": chunk_ms + union_ms + attend_union_dense_ms,
+                  "group_attend_eps0_ms": group_dense_ms, "group_attend_eps_ms": group_eps_ms,
+                  "step_eps0_ms": chunk_ms + union_ms + min(attend_union_dense_ms, group_dense_ms),
                   "err_eps0_vs_dense": err(union_dense_out)},
         "pool_bytes": {"full": full_bytes, "chunk": chunk_bytes},
         "dense_causal_tflop": wl.dense_causal_flops() / 1e12,
@@ -568,10 +580,34 @@ def main():
             b.record(stream)
             torch.cuda.synchronize()
         dense_ms = max_over_ranks([a.elapsed_time(b) / dsteps], dist, dev)[0]
-        dense = {"ms": dense_ms, "tflops": dense_flops / (dense_ms * 1e-3) / 1e12,
+        dense = {"kernel": "osk_attention", "ms": dense_ms, "tflops": dense_flops / (dense_ms * 1e-3) / 1e12,
                  "frac_of_peak": dense_flops / (dense_ms * 1e-3) / 1e12 / tc_peak,
                  "speedup_of_sparse_step": dense_ms / ms_step, "clocks": dclk.summary()}
         del d_order, d_count
+        if (wl.Hq // wl.Hkv) % 2 == 0:
+            # the same dense path through the group kernel (one order per
+            # kv-head group, each K/V tile loaded once for two query heads);
+            # the dense path reported is the faster of the two
+            g_order, g_count = m.dense_order_group()
+            m.attend_group(q, k, v, g_order, g_count, 0.0, page_table=pt, out=out)
+            torch.cuda.synchronize()
+            a, b = ev(), ev()
+            with ClockSampler(local) as gclk:
+                a.record(stream)
+                for _ in range(dsteps):
+                    cosa.cosa_attend_group(shape, q, k, v, pt, g_order, g_count, g_order.shape[-1], 0.0, out, None,
+                                           None, m.status, stream)
+                b.record(stream)
+                torch.cuda.synchronize()
+            g_ms = max_over_ranks([a.elapsed_time(b) / dsteps], dist, dev)[0]
+            group = {"kernel": "osk_group", "ms": g_ms, "tflops": dense_flops / (g_ms * 1e-3) / 1e12,
+                     "frac_of_peak": dense_flops / (g_ms * 1e-3) / 1e12 / tc_peak,
+                     "speedup_of_sparse_step": g_ms / ms_step, "clocks": gclk.summary()}
+            per_head = dict(dense)
+            dense = dict(group if g_ms < dense_ms else per_head)
+            dense["per_head_kernel"] = {k_: per_head[k_] for k_ in ("ms", "tflops", "frac_of_peak")}
+            dense["group_kernel"] = {k_: group[k_] for k_ in ("ms", "tflops", "frac_of_peak")}
+            del g_order, g_count
         # context only, not this library: torch's fused causal attention on the
         # same inputs (whatever backend torch picks), when its top-left causal
         # alignment matches (Nq == Nkv) and K/V are contiguous

@@ -62,6 +62,7 @@ _lib.cosa_decode_plan.argtypes = [_S, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int
                                   _P, _P, _P, _P, _P, _P]
 _lib.cosa_plan_static.argtypes = [_S, _P, _P, _P, ctypes.c_double, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P]
 _lib.cosa_attend.argtypes = [_S, _P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_double, _P, _P, _P, _P, _P]
+_lib.cosa_attend_group.argtypes = [_S, _P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_double, _P, _P, _P, _P, _P]
 _lib.cosa_test_attend_wait_timeout.argtypes = [_S, _P, _P, _P, _P, _P, _P, ctypes.c_int, _P, _P, ctypes.c_uint64, _P]
 _lib.cosa_skip_threshold.argtypes = [ctypes.c_double, ctypes.c_int]
 _lib.cosa_skip_threshold.restype = ctypes.c_float
@@ -71,7 +72,7 @@ _lib.cosa_status_string.restype = ctypes.c_char_p
 EXPORTS = ("cosa_num_qblocks", "cosa_num_kblocks", "cosa_kmax", "cosa_plan_workspace_bytes", "cosa_plan",
            "cosa_dense_order", "cosa_attend", "cosa_skip_threshold", "cosa_status_string", "cosa_version",
            "cosa_plan_static", "cosa_plan_chunk", "cosa_block_union", "cosa_decode_plan",
-           "cosa_test_attend_wait_timeout")
+           "cosa_test_attend_wait_timeout", "cosa_attend_group")
 DEV_TIMEOUT_TMA, DEV_TIMEOUT_MMA, DEV_TIMEOUT_PIPE = 0x100, 0x200, 0x300
 STATIC_SCRATCH_BYTES = 64 << 20
 
@@ -222,6 +223,19 @@ def cosa_attend(shape: cosa_shape, q, k, v, page_table, order, count, kmax: int,
                             _stream(stream)), "cosa_attend")
 
 
+def cosa_attend_group(shape: cosa_shape, q, k, v, page_table, order, count, kmax: int, skip_eps: float, out,
+                      lse=None, skip_bits=None, dev_status=None, stream=None) -> None:
+    """OSK with one visit order per (batch, kv-head, Q-block) shared by the
+    group's query heads: order [B, Hkv, nQB, kmax], count [B, Hkv, nQB]."""
+    _check(_lib.cosa_attend_group(ctypes.byref(shape), _ptr(q, "q", torch.bfloat16), _ptr(k, "k", torch.bfloat16),
+                                  _ptr(v, "v", torch.bfloat16), _ptr(page_table, "page_table", torch.int32),
+                                  _ptr(order, "order", torch.int32), _ptr(count, "count", torch.int32), kmax,
+                                  skip_eps, _ptr(out, "out", torch.bfloat16), _ptr(lse, "lse", torch.float32),
+                                  _ptr(skip_bits, "skip_bits", torch.int32),
+                                  _ptr(dev_status, "dev_status", torch.int32), _stream(stream)),
+           "cosa_attend_group")
+
+
 def cosa_test_attend_wait_timeout(shape: cosa_shape, q, k, v, page_table, order, count, kmax: int, out,
                                   dev_status, wait_limit_ns: int, stream=None) -> None:
     """Failure-detection test hook: cosa_attend's kernel with one wait per
@@ -354,9 +368,37 @@ class CoSA:
         cosa_attend(s, q, k, v, page_table, order, count, km, eps, out, lse_t, sb, self.status, stream)
         return dict(out=out, lse=lse_t, skip_bits=sb)
 
-    def dense(self, q, k, v, page_table=None, stream=None, **kw):
+    def dense(self, q, k, v, page_table=None, stream=None, group: bool = False, **kw):
+        """The dense path: every causal block, eps 0.  group=True runs it
+        through attend_group (one shared order per GQA group)."""
+        if group:
+            order, count = self.dense_order_group(stream)
+            return self.attend_group(q, k, v, order, count, 0.0, page_table=page_table, stream=stream, **kw)
         order, count = self.dense_order(stream)
         return self.attend(q, k, v, order, count, 0.0, page_table=page_table, stream=stream, **kw)
+
+    def dense_order_group(self, stream=None):
+        """The dense path's order with one row per (b, kv-head, Q-block)."""
+        s = self.shape
+        gs = make_shape(s.B, s.Hkv, s.Hkv, s.Nq, s.Nkv, s.d, s.bq, s.bk, s.stride, bool(s.paged), s.num_pages)
+        order = torch.empty(s.B, s.Hkv, self.nqb, self.nkb, dtype=torch.int32, device=self.device)
+        count = torch.empty(s.B, s.Hkv, self.nqb, dtype=torch.int32, device=self.device)
+        cosa_dense_order(gs, self.nkb, order, count, stream)
+        return order, count
+
+    def attend_group(self, q, k, v, order, count, eps: float, page_table=None, out=None, lse: bool = False,
+                     skip_bits: bool = False, stream=None):
+        """attend() with one order per (b, kv-head, Q-block): order
+        [B, Hkv, nQB, kmax], count [B, Hkv, nQB]."""
+        s = self.shape
+        km = order.shape[-1]
+        if out is None:
+            out = torch.empty(s.B, s.Hq, s.Nq, s.d, dtype=torch.bfloat16, device=self.device)
+        lse_t = torch.empty(s.B, s.Hq, s.Nq, dtype=torch.float32, device=self.device) if lse else None
+        sb = torch.empty(s.B, s.Hq, self.nqb, (km + 31) // 32, dtype=torch.int32, device=self.device) \
+            if skip_bits else None
+        cosa_attend_group(s, q, k, v, page_table, order, count, km, eps, out, lse_t, sb, self.status, stream)
+        return dict(out=out, lse=lse_t, skip_bits=sb)
 
     def device_status(self) -> int:
         return int(self.status.item())

@@ -361,7 +361,7 @@ namespace {
 cosa_status attend_impl(const cosa_shape* shape, const void* q, const void* k, const void* v,
                         const int32_t* page_table, const int32_t* order, const int32_t* count, int kmax,
                         double skip_eps, void* out, float* lse, uint32_t* skip_bits, uint32_t* dev_status,
-                        uint64_t wait_limit_ns, int stall_test, cudaStream_t stream) {
+                        uint64_t wait_limit_ns, int stall_test, bool group, cudaStream_t stream) {
   cosa_status st = check_shape(shape);
   if (st != COSA_OK) return st;
   if (!(skip_eps >= 0.0) || skip_eps >= 1.0) return COSA_EINVAL;
@@ -387,6 +387,7 @@ cosa_status attend_impl(const cosa_shape* shape, const void* q, const void* k, c
   p.status = dev_status;
   p.wait_limit_ns = wait_limit_ns;
   p.stall_test = stall_test;
+  if (group) return launch_status(launch_osk_group(tm_q, tm_k, tm_v, p, s.bk, stream));
   return launch_status(launch_osk(tm_q, tm_k, tm_v, p, s.bk, stream));
 }
 
@@ -399,7 +400,23 @@ cosa_status cosa_attend(const cosa_shape* shape, const void* q, const void* k, c
                         double skip_eps, void* out, float* lse, uint32_t* skip_bits, uint32_t* dev_status,
                         cudaStream_t stream) {
   return attend_impl(shape, q, k, v, page_table, order, count, kmax, skip_eps, out, lse, skip_bits, dev_status,
-                     1000000000ull, 0, stream);
+                     1000000000ull, 0, false, stream);
+}
+
+cosa_status cosa_attend_group(const cosa_shape* shape, const void* q, const void* k, const void* v,
+                              const int32_t* page_table, const int32_t* order, const int32_t* count, int kmax,
+                              double skip_eps, void* out, float* lse, uint32_t* skip_bits, uint32_t* dev_status,
+                              cudaStream_t stream) {
+  cosa_status st = check_shape(shape);
+  if (st != COSA_OK) return st;
+  const int G = shape->Hq / shape->Hkv;
+  // one query head per group: the group's order is the head's order
+  if (G == 1)
+    return attend_impl(shape, q, k, v, page_table, order, count, kmax, skip_eps, out, lse, skip_bits, dev_status,
+                       1000000000ull, 0, false, stream);
+  if (G % 2) return COSA_EUNSUPPORTED;
+  return attend_impl(shape, q, k, v, page_table, order, count, kmax, skip_eps, out, lse, skip_bits, dev_status,
+                     1000000000ull, 0, true, stream);
 }
 
 cosa_status cosa_test_attend_wait_timeout(const cosa_shape* shape, const void* q, const void* k, const void* v,
@@ -408,7 +425,7 @@ cosa_status cosa_test_attend_wait_timeout(const cosa_shape* shape, const void* q
                                           cudaStream_t stream) {
   if (!dev_status || wait_limit_ns < 1000ull || wait_limit_ns > 1000000000ull) return COSA_EINVAL;
   return attend_impl(shape, q, k, v, page_table, order, count, kmax, 0.0, out, nullptr, nullptr, dev_status,
-                     wait_limit_ns, 1, stream);
+                     wait_limit_ns, 1, false, stream);
 }
 
 const char* cosa_status_string(cosa_status status) {

@@ -96,5 +96,9 @@ struct OskParams {
 };
 cudaError_t launch_osk(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                        const OskParams& p, int bk, cudaStream_t st);
+// The same with one order per (b, kv-head, Q-block) shared by the G query
+// heads (order [B, Hkv, nQB, kmax], count [B, Hkv, nQB]); G even.
+cudaError_t launch_osk_group(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                             const OskParams& p, int bk, cudaStream_t st);
 
 }  // namespace cosa

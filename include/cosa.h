@@ -215,6 +215,29 @@ COSA_API cosa_status cosa_attend(const cosa_shape* shape, const void* q, const v
                         double skip_eps, void* out, float* lse, uint32_t* skip_bits, uint32_t* dev_status,
                         cudaStream_t stream);
 
+/* OSK over one visit order per GQA group: the execution form of
+ * "CompactAttention: Accelerating Chunked Prefill with Block-Union KV
+ * Selection" (method, execution stage: one block table per (batch, kv-head
+ * group), read in place), run with CoSA's ordered skipping (technical
+ * summary Sec. 2.3).  Every query head of kv-head g visits the blocks
+ * order[b,g,I,0..count-1] in that order; per head the arithmetic, the skip
+ * vote (on that head's own 128-row tile) and the results are exactly those
+ * of cosa_attend given the same order for each head of the group, but each
+ * K/V tile is loaded once for two heads.
+ *  order      [B, Hkv, nQB, kmax] int32 in (cosa_block_union's union_order
+ *             rows are the same for every head of a group: any one of them
+ *             serves; cosa_dense_order on a shape with Hq = Hkv gives the
+ *             dense path's).
+ *  count      [B, Hkv, nQB] int32 in.
+ *  out, lse, skip_bits, dev_status: as for cosa_attend (per query head).
+ * Returns COSA_EUNSUPPORTED when Hq / Hkv is odd and above 1 (G = 1 runs
+ * cosa_attend's kernel, whose order layout is then the same), and otherwise
+ * what cosa_attend returns for the same arguments. */
+COSA_API cosa_status cosa_attend_group(const cosa_shape* shape, const void* q, const void* k, const void* v,
+                                       const int32_t* page_table, const int32_t* order, const int32_t* count,
+                                       int kmax, double skip_eps, void* out, float* lse, uint32_t* skip_bits,
+                                       uint32_t* dev_status, cudaStream_t stream);
+
 /* Failure-detection test hook (no counterpart in the papers): runs
  * cosa_attend's kernel with skip_eps = 0 on the given arguments, except that
  * in every CTA the issuing thread, before the first QK^T, waits on a barrier
