@@ -121,12 +121,15 @@ osk_group_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       auto slot_addr = [&](int sl) { return sl ? v_addr : k_addr; };
       uint32_t fph = 0u;     // bit sl: parity of the next completion to wait for on slot sl
       uint32_t busy = 0u;    // bit sl: a load into slot sl was issued and not yet seen complete
+      // K/V tiles are read again soon by the other heads of the group and by
+      // neighbouring Q-blocks: keep them in L2; each Q tile is read once
+      const uint64_t pol_kv = l2_evict_last(), pol_q = l2_evict_first();
       auto load = [&](int sl, const CUtensorMap* tm, int j) {
         const int y = kv_row<BK>(p, b, g, j);
         busy |= 1u << sl;
         mbar_arrive_expect_tx(&sm->full[sl], Cfg::kKVBytes);
-        tma_load_2d(slot(sl), tm, &sm->full[sl], 0, y);
-        tma_load_2d(slot(sl) + Cfg::kChunk, tm, &sm->full[sl], 64, y);
+        tma_load_2d_hint(slot(sl), tm, &sm->full[sl], 0, y, pol_kv);
+        tma_load_2d_hint(slot(sl) + Cfg::kChunk, tm, &sm->full[sl], 64, y, pol_kv);
       };
       auto wait_slot = [&](int sl) {
         const bool r = wait_or_abort(&sm->full[sl], (fph >> sl) & 1u, abort, p.status, DEV_TIMEOUT_TMA,
@@ -148,8 +151,8 @@ osk_group_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       mbar_arrive_expect_tx(&sm->q_full, kHeads * kQBytes);
       for (int hh = 0; hh < kHeads; ++hh) {
         const int q_y = (b * p.Hq + h0 + hh) * p.Nq + I * p.bq;
-        tma_load_2d(sQ + hh * kQBytes, &tm_q, &sm->q_full, 0, q_y);
-        tma_load_2d(sQ + hh * kQBytes + 16384, &tm_q, &sm->q_full, 64, q_y);
+        tma_load_2d_hint(sQ + hh * kQBytes, &tm_q, &sm->q_full, 0, q_y, pol_q);
+        tma_load_2d_hint(sQ + hh * kQBytes + 16384, &tm_q, &sm->q_full, 64, q_y, pol_q);
       }
       load(0, &tm_k, order_at(0));
       if (n > 1) load(1, &tm_k, order_at(1));
