@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--heads", default=None, metavar="HQ:HKV",
                     help="override the workload's query/kv head counts (a smaller case of the same layer, "
                          "e.g. for profiling); the workload is then reported as NAME[hqHQ:hkvHKV]")
+    ap.add_argument("--recipe", default="default", choices=["default", "planned"],
+                    help="input recipe: the default one, or the first plan's weaker structure")
     ap.add_argument("--budget", type=float, default=None)
     ap.add_argument("--eps", type=float, default=None)
     ap.add_argument("--impl", default="cosa", choices=["cosa", "reference"])
@@ -393,9 +395,11 @@ def run_decode(args, wl, budget, eps):
     """One decode step: the last query row of every head of the workload is
     the new token (position Nkv-1); the pooled keys are already cached, as
     after a prefill with cosa_plan_chunk.  Times the proxy (cosa_decode_plan)
-    and the attention (cosa_attend with Nq = 1), against the dense decode
-    step (every block, eps 0) on the same kernel; reports the K/V bytes the
-    sparse step reads and its error against the dense step."""
+    and the attention (cosa_decode_attend), against the dense decode step
+    (every block, eps 0) on the same kernels; reports the K/V bytes the
+    sparse step reads, the rate at which it reads them against the measured
+    HBM bandwidth, and its error against the dense step.  cosa_attend on the
+    same one-row shape is timed as context."""
     import block_sparse_attention_kap_b200 as cosa
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(dev)
@@ -428,13 +432,20 @@ def run_decode(args, wl, budget, eps):
 
     plan_ms = timed(lambda: cosa.cosa_decode_plan(shape, q, k, pt, cache, nkp, budget, km, order, count,
                                                   plan["hrm_count"], None, None, stream))
-    attend_ms = timed(lambda: cosa.cosa_attend(shape, q, k, v, pt, order, count, km, eps, out, None, None,
-                                               m.status, stream))
+    tile_attend_ms = timed(lambda: cosa.cosa_attend(shape, q, k, v, pt, order, count, km, eps, out, None, None,
+                                                    m.status, stream))
     d_order, d_count = m.dense_order()
-    dense_ms = timed(lambda: cosa.cosa_attend(shape, q, k, v, pt, d_order, d_count, d_order.shape[-1], 0.0, out,
-                                              None, None, m.status, stream))
-    res = m.attend(q, k, v, order, count, eps, page_table=pt, skip_bits=True)
-    dense_out = m.attend(q, k, v, d_order, d_count, 0.0, page_table=pt)["out"].float()
+    d_km = d_order.shape[-1]
+    ws = torch.empty(max(cosa.cosa_decode_attend_workspace_bytes(shape, km),
+                         cosa.cosa_decode_attend_workspace_bytes(shape, d_km)), dtype=torch.uint8, device=dev)
+    attend_ms = timed(lambda: cosa.cosa_decode_attend(shape, q, k, v, pt, order, count, km, eps, out, None, None,
+                                                      ws, stream))
+    dense_ms = timed(lambda: cosa.cosa_decode_attend(shape, q, k, v, pt, d_order, d_count, d_km, 0.0, out, None,
+                                                     None, ws, stream))
+    tile_dense_ms = timed(lambda: cosa.cosa_attend(shape, q, k, v, pt, d_order, d_count, d_km, 0.0, out, None, None,
+                                                   m.status, stream))
+    res = m.decode_attend(q, k, v, order, count, eps, page_table=pt, skip_bits=True)
+    dense_out = m.decode_attend(q, k, v, d_order, d_count, 0.0, page_table=pt)["out"].float()
     torch.cuda.synchronize()
     assert m.device_status() == 0
     sel = int(count.sum().item())
@@ -444,13 +455,19 @@ def run_decode(args, wl, budget, eps):
     dense_bytes = 2 * tile * int(d_count.sum().item())
     err = (res["out"].float() - dense_out).abs()
     rows = wl.B * wl.Hq
+    hbm_peak = load_peaks()[0]
     print(json.dumps({
         "kind": "decode", "workload": wl.name, "rows": rows, "Nkv": wl.Nkv, "budget": budget, "eps": eps,
         "plan_ms": plan_ms, "attend_ms": attend_ms, "step_ms": plan_ms + attend_ms, "dense_step_ms": dense_ms,
         "speedup_vs_dense": dense_ms / (plan_ms + attend_ms),
         "selected_blocks": sel, "skipped_in_kernel_frac": skipped / max(1, sel),
         "kv_bytes": {"sparse": sparse_bytes, "dense": dense_bytes},
-        "attend_gbs_requested": sparse_bytes / (attend_ms * 1e-3) / 1e9,
+        "attend_gbs": sparse_bytes / (attend_ms * 1e-3) / 1e9,
+        "attend_frac_of_hbm": sparse_bytes / (attend_ms * 1e-3) / 1e9 / hbm_peak,
+        "dense_gbs": dense_bytes / (dense_ms * 1e-3) / 1e9,
+        "dense_frac_of_hbm": dense_bytes / (dense_ms * 1e-3) / 1e9 / hbm_peak,
+        "tile_kernel_context": {"attend_ms": tile_attend_ms, "dense_ms": tile_dense_ms,
+                                "note": "cosa_attend (128-row tensor-core tiles, one valid row) on the same step"},
         "err_vs_dense": {"max_abs": err.max().item(), "mean_abs": err.mean().item()}}), flush=True)
 
 
@@ -462,6 +479,8 @@ def main():
     if args.heads:
         hq, hkv = (int(x) for x in args.heads.split(":"))
         wl = wl.replace(Hq=hq, Hkv=hkv, name=f"{wl.name}[hq{hq}:hkv{hkv}]")
+    if args.recipe != "default":
+        wl = wl.replace(recipe=args.recipe, name=f"{wl.name}[{args.recipe}]")
     budget = args.budget if args.budget is not None else (0.1 if 0.1 in wl.budgets else wl.budgets[0])
     eps = args.eps if args.eps is not None else wl.eps
     if args.impl == "reference":

@@ -62,6 +62,10 @@ _lib.cosa_decode_plan.argtypes = [_S, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int
                                   _P, _P, _P, _P, _P, _P]
 _lib.cosa_plan_static.argtypes = [_S, _P, _P, _P, ctypes.c_double, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P]
 _lib.cosa_attend.argtypes = [_S, _P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_double, _P, _P, _P, _P, _P]
+_lib.cosa_decode_attend_workspace_bytes.argtypes = [_S, ctypes.c_int]
+_lib.cosa_decode_attend_workspace_bytes.restype = ctypes.c_size_t
+_lib.cosa_decode_attend.argtypes = [_S, _P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_double, _P, _P, _P, _P,
+                                    ctypes.c_size_t, _P]
 _lib.cosa_attend_group.argtypes = [_S, _P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_double, _P, _P, _P, _P, _P]
 _lib.cosa_test_attend_wait_timeout.argtypes = [_S, _P, _P, _P, _P, _P, _P, ctypes.c_int, _P, _P, ctypes.c_uint64, _P]
 _lib.cosa_skip_threshold.argtypes = [ctypes.c_double, ctypes.c_int]
@@ -72,7 +76,8 @@ _lib.cosa_status_string.restype = ctypes.c_char_p
 EXPORTS = ("cosa_num_qblocks", "cosa_num_kblocks", "cosa_kmax", "cosa_plan_workspace_bytes", "cosa_plan",
            "cosa_dense_order", "cosa_attend", "cosa_skip_threshold", "cosa_status_string", "cosa_version",
            "cosa_plan_static", "cosa_plan_chunk", "cosa_block_union", "cosa_decode_plan",
-           "cosa_test_attend_wait_timeout", "cosa_attend_group")
+           "cosa_test_attend_wait_timeout", "cosa_attend_group", "cosa_decode_attend",
+           "cosa_decode_attend_workspace_bytes")
 DEV_TIMEOUT_TMA, DEV_TIMEOUT_MMA, DEV_TIMEOUT_PIPE = 0x100, 0x200, 0x300
 STATIC_SCRATCH_BYTES = 64 << 20
 
@@ -223,6 +228,24 @@ def cosa_attend(shape: cosa_shape, q, k, v, page_table, order, count, kmax: int,
                             _stream(stream)), "cosa_attend")
 
 
+def cosa_decode_attend_workspace_bytes(shape: cosa_shape, kmax: int) -> int:
+    return _lib.cosa_decode_attend_workspace_bytes(ctypes.byref(shape), kmax)
+
+
+def cosa_decode_attend(shape: cosa_shape, q, k, v, page_table, order, count, kmax: int, skip_eps: float, out,
+                       lse=None, skip_bits=None, workspace=None, stream=None) -> None:
+    """The attention of one decode step (shape.Nq == 1): OSK on the single
+    query row of each head, with memory-bound kernels (parallel logits, a
+    prefix-max scan for the skip decisions, parallel P.V)."""
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.cosa_decode_attend(ctypes.byref(shape), _ptr(q, "q", torch.bfloat16), _ptr(k, "k", torch.bfloat16),
+                                   _ptr(v, "v", torch.bfloat16), _ptr(page_table, "page_table", torch.int32),
+                                   _ptr(order, "order", torch.int32), _ptr(count, "count", torch.int32), kmax,
+                                   skip_eps, _ptr(out, "out", torch.bfloat16), _ptr(lse, "lse", torch.float32),
+                                   _ptr(skip_bits, "skip_bits", torch.int32), _ptr(workspace, "workspace"), ws_bytes,
+                                   _stream(stream)), "cosa_decode_attend")
+
+
 def cosa_attend_group(shape: cosa_shape, q, k, v, page_table, order, count, kmax: int, skip_eps: float, out,
                       lse=None, skip_bits=None, dev_status=None, stream=None) -> None:
     """OSK with one visit order per (batch, kv-head, Q-block) shared by the
@@ -334,6 +357,22 @@ class CoSA:
         if scores:
             res.update(block_score=bs, hrm=hf)
         return res
+
+    def decode_attend(self, q, k, v, order, count, eps: float, page_table=None, out=None, lse: bool = False,
+                      skip_bits: bool = False, stream=None):
+        """The attention of one decode step (shape.Nq == 1) with the decode
+        kernels: order [B, Hq, 1, kmax], count [B, Hq, 1]."""
+        s = self.shape
+        km = order.shape[-1]
+        if out is None:
+            out = torch.empty(s.B, s.Hq, 1, s.d, dtype=torch.bfloat16, device=self.device)
+        lse_t = torch.empty(s.B, s.Hq, 1, dtype=torch.float32, device=self.device) if lse else None
+        sb = torch.empty(s.B, s.Hq, 1, (km + 31) // 32, dtype=torch.int32, device=self.device) if skip_bits else None
+        nbytes = cosa_decode_attend_workspace_bytes(s, km)
+        if getattr(self, "_dws", None) is None or self._dws.numel() < nbytes:
+            self._dws = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        cosa_decode_attend(s, q, k, v, page_table, order, count, km, eps, out, lse_t, sb, self._dws, stream)
+        return dict(out=out, lse=lse_t, skip_bits=sb)
 
     def block_union(self, order, count, expand: bool = True, stream=None):
         """Per-(batch, kv-head) union of a selection over the Q-blocks and the

@@ -331,6 +331,42 @@ cosa_status cosa_decode_plan(const cosa_shape* shape, const void* q, const void*
   return launch_status(launch_decode_plan(dp, stream));
 }
 
+size_t cosa_decode_attend_workspace_bytes(const cosa_shape* shape, int kmax) {
+  if (check_shape(shape) != COSA_OK || shape->Nq != 1 || kmax < 1) return 0;
+  return decode_attend_workspace(shape->B * shape->Hq, kmax, shape->bk);
+}
+
+cosa_status cosa_decode_attend(const cosa_shape* shape, const void* q, const void* k, const void* v,
+                               const int32_t* page_table, const int32_t* order, const int32_t* count, int kmax,
+                               double skip_eps, void* out, float* lse, uint32_t* skip_bits, void* workspace,
+                               size_t ws_bytes, cudaStream_t stream) {
+  cosa_status st = check_shape(shape);
+  if (st != COSA_OK) return st;
+  const cosa_shape& s = *shape;
+  if (s.Nq != 1) return COSA_ESHAPE;
+  if (!(skip_eps >= 0.0) || skip_eps >= 1.0) return COSA_EINVAL;
+  const int rows = s.B * s.Hq;
+  if (rows == 0) return COSA_OK;
+  if (!q || !k || !v || !out || !order || !count || (s.paged && !page_table)) return COSA_EINVAL;
+  if (kmax < 1) return COSA_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return COSA_EALIGN;
+  if (decode_attend_smem(kmax, s.bk) > 227 * 1024) return COSA_EUNSUPPORTED;
+  if (!workspace || ws_bytes < decode_attend_workspace(rows, kmax, s.bk)) return COSA_EWORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255) return COSA_EALIGN;
+  DecodeAttendParams p;
+  p.B = s.B; p.Hq = s.Hq; p.Hkv = s.Hkv; p.Nkv = s.Nkv; p.nkb = n_kblocks(&s); p.bk = s.bk;
+  p.paged = s.paged; p.num_pages = s.num_pages; p.kmax = kmax;
+  p.q = static_cast<const uint16_t*>(q);
+  p.k = static_cast<const uint16_t*>(k);
+  p.v = static_cast<const uint16_t*>(v);
+  p.page_table = page_table; p.order = order; p.count = count;
+  p.T = cosa_skip_threshold(skip_eps, s.d);
+  p.scale_ln = (float)(1.0 / std::sqrt((double)s.d));
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)s.d));
+  p.out = static_cast<uint16_t*>(out); p.lse = lse; p.skip_bits = skip_bits; p.skip_words = cdiv(kmax, 32);
+  return launch_status(launch_decode_attend(p, static_cast<uint8_t*>(workspace), stream));
+}
+
 cosa_status cosa_block_union(const cosa_shape* shape, const int32_t* order, const int32_t* count, int kmax,
                              int32_t* table, int32_t* table_len, int32_t* union_order, int32_t* union_count,
                              int union_kmax, cudaStream_t stream) {

@@ -11,11 +11,16 @@
 // and the blocks are ordered HRM first, then by z, ties by block index, the
 // first k = max(1, ceil(nKB * budget)) kept (warp_select_sort).
 //
-// One CTA (8 warps) per (b, h).  Warp w scores blocks w, w+8, ...: eight
-// lanes per pooled key (16 bf16 dimensions each, two 16-byte loads), four
-// keys per step, a three-step shuffle sum, a running max per block.  The
-// block scores stay in shared memory; a CTA-wide arg-max, the keys, and one
-// warp's select-and-sort follow.
+// One cluster of kCluster CTAs (8 warps each) per (b, h): CTA r of the
+// cluster scores the r-th contiguous share of the blocks -- warp w its
+// blocks w, w+8, ...: eight lanes per pooled key (16 bf16 dimensions each,
+// two 16-byte loads), four keys per step, a three-step shuffle sum, a
+// running max per block -- and stores each block score straight into the
+// shared memory of CTA 0 of the cluster (distributed shared memory).  After
+// a cluster barrier CTA 0 alone holds every block score: a CTA-wide arg-max,
+// the keys, and one warp's select-and-sort follow.  Splitting the scoring
+// over the cluster puts eight times as many warps on the pooled-key reads,
+// which are latency-bound at one CTA per head.
 #include "kap_select.cuh"
 #include "decode.h"
 
@@ -24,11 +29,28 @@ namespace cosa {
 namespace {
 
 constexpr int kWarps = 8;
+constexpr int kCluster = 8;                   // CTAs per (b, h)
+
+// Store v at the same shared-memory offset as `local` in CTA `rank` of the cluster.
+__device__ __forceinline__ void st_cluster_f32(const float* local, uint32_t rank, float v) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote)
+               : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(local))), "r"(rank));
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-__global__ void __launch_bounds__(32 * kWarps) decode_plan_kernel(DecodePlanParams p) {
+__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(32 * kWarps) decode_plan_kernel(DecodePlanParams p) {
   extern __shared__ __align__(16) uint8_t dyn[];
   float* bs = reinterpret_cast<float*>(dyn);                               // [nkb] block scores, then keys
   int* hist = reinterpret_cast<int*>(dyn + align16((size_t)p.nkb * 4));
@@ -36,7 +58,10 @@ __global__ void __launch_bounds__(32 * kWarps) decode_plan_kernel(DecodePlanPara
   __shared__ float red_m[kWarps];
   __shared__ int red_j[kWarps];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int hb = blockIdx.x;                                               // b * Hq + h
+  const int hb = blockIdx.x / kCluster;                                   // b * Hq + h
+  const uint32_t rank = cluster_rank();
+  const int per = (p.nkb + kCluster - 1) / kCluster;                       // this CTA's blocks: [j0, j1)
+  const int j0 = min(p.nkb, (int)rank * per), j1 = min(p.nkb, j0 + per);
   const int b = hb / p.Hq, h = hb - b * p.Hq;
   const int g = h / (p.Hq / p.Hkv);
   const int grp = lane >> 3, part = lane & 7;                              // key within the step, 16-dim slice
@@ -51,7 +76,8 @@ __global__ void __launch_bounds__(32 * kWarps) decode_plan_kernel(DecodePlanPara
     for (int i = 0; i < 8; ++i) { qf[2 * i] = bf16_lo(w[i]); qf[2 * i + 1] = bf16_hi(w[i]); }
   }
   const uint16_t* kp = p.kp + ((size_t)b * p.Hkv + g) * (size_t)p.kp_stride * kD;
-  for (int j = warp; j < p.nkb; j += kWarps) {
+  cluster_sync();                     // every CTA of the cluster runs before any remote store
+  for (int j = j0 + warp; j < j1; j += kWarps) {
     float m = -INFINITY;
     const int c0 = j * p.kpb, c1 = min(c0 + p.kpb, p.nkp);
     const int steps = (c1 - c0 + 3) / 4;                                // every lane runs every step
@@ -74,9 +100,10 @@ __global__ void __launch_bounds__(32 * kWarps) decode_plan_kernel(DecodePlanPara
     }
 #pragma unroll
     for (int o = 8; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) bs[j] = m;
+    if (lane == 0) st_cluster_f32(bs + j, 0u, m);                          // into CTA 0's block scores
   }
-  __syncthreads();
+  cluster_sync();                                                          // every score is in CTA 0
+  if (rank != 0) return;
 
   // CTA-wide maximum and the first block attaining it
   float m = -INFINITY;
@@ -132,7 +159,7 @@ cudaError_t launch_decode_plan(const DecodePlanParams& p, cudaStream_t st) {
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(decode_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  decode_plan_kernel<<<rows, 32 * kWarps, smem, st>>>(p);
+  decode_plan_kernel<<<rows * kCluster, 32 * kWarps, smem, st>>>(p);
   return cudaGetLastError();
 }
 

@@ -11,10 +11,9 @@
 // maxima come from kap_score's per-item partial maxima (ties resolved to the
 // smaller block index).  Each block's ranking key (+1 for HRM blocks, else
 // its score <= 0) is mapped to an order-preserving 32-bit integer, and
-// warp_select_sort (kap_select.cuh) emits the order.  Used by kap_sort (a
-// kernel of its own) and by the last work item of each row tile in
-// kap_score; Bs and the partial maxima are read through L2 (ld.global.cg),
-// since in the second case other CTAs of the same launch wrote them.
+// warp_select_sort (kap_select.cuh) emits the order.  Used by kap_sort, one
+// warp per (b, h, Q-block); Bs and the partial maxima come from the
+// preceding kap_score launch and are read through the read-only path.
 #pragma once
 #include "kap_select.cuh"
 
@@ -47,8 +46,8 @@ __device__ __forceinline__ void rank_qblock(const SortParams& p, int row, int pk
   if (lane < RPQ) {
     const size_t base = ((size_t)hb * p.n_row_tiles + R) * p.splits * 2 * kTileRows + row0 + lane;
     for (int q = 0; q < 2 * p.splits; ++q) {
-      const float m = __ldcg(p.part_max + base + (size_t)q * kTileRows);
-      const int a = __ldcg(p.part_arg + base + (size_t)q * kTileRows);
+      const float m = __ldg(p.part_max + base + (size_t)q * kTileRows);
+      const int a = __ldg(p.part_arg + base + (size_t)q * kTileRows);
       if (m > my_max || (m == my_max && a >= 0 && (my_arg < 0 || a < my_arg))) { my_max = m; my_arg = a; }
     }
   }
@@ -71,12 +70,12 @@ __device__ __forceinline__ void rank_qblock(const SortParams& p, int row, int pk
     if constexpr (RPQ % 4 == 0) {
 #pragma unroll
       for (int i = 0; i < RPQ; i += 4) {
-        const float4 f = __ldcg(reinterpret_cast<const float4*>(src + i));
+        const float4 f = __ldg(reinterpret_cast<const float4*>(src + i));
         v[i] = f.x; v[i + 1] = f.y; v[i + 2] = f.z; v[i + 3] = f.w;
       }
     } else {
 #pragma unroll
-      for (int i = 0; i < RPQ; ++i) v[i] = __ldcg(src + i);
+      for (int i = 0; i < RPQ; ++i) v[i] = __ldg(src + i);
     }
     float z = -INFINITY;
     bool flag = false;

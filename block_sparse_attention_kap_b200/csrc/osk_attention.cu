@@ -197,13 +197,18 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           const int valid = (jv >= 0 && jv < p.nkb) ? min(BK, p.Nkv - jv * BK) : BK;   // >= 1
           const int ksteps = clear_v_tail(slot(ks), Cfg::kChunk, valid);
           tc_fence_after();
+          // P of keys [16kk, 16kk+16): each column half packs its P at the
+          // start of its own S range (TMEM columns half*BK/2 + ...)
+          auto pv_step = [&](int kk) {
+            mma_ts(tO, tS + (kk / (BK / 32)) * (BK / 2) + (kk % (BK / 32)) * 8,
+                   desc_sw128(slot_addr(ks) + kk * 2048, Cfg::kChunk, 1024), id_pv, (any_pv || kk > 0) ? 1u : 0u);
+          };
+          if (ksteps == BK / 16) {
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            // P of keys [16kk, 16kk+16): each column half packs its P at the
-            // start of its own S range (TMEM columns half*BK/2 + ...)
-            if (kk < ksteps)
-              mma_ts(tO, tS + (kk / (BK / 32)) * (BK / 2) + (kk % (BK / 32)) * 8,
-                     desc_sw128(slot_addr(ks) + kk * 2048, Cfg::kChunk, 1024), id_pv, (any_pv || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < BK / 16; ++kk) pv_step(kk);
+          } else {
+            for (int kk = 0; kk < ksteps; ++kk) pv_step(kk);
+          }
           any_pv = true;
           if (t + 2 < n) pend_k = t + 2;
         }

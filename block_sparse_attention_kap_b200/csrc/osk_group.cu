@@ -205,14 +205,19 @@ osk_group_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
               v_seen = true;
             }
             tc_fence_after();
+            // P of keys [16kk, 16kk+16): each column half of the head's S
+            // range holds its P at the start of that half
+            auto pv_step = [&](int kk) {
+              mma_ts(tO(hh), tS(hh) + (kk / (BK / 32)) * (BK / 2) + (kk % (BK / 32)) * 8,
+                     desc_sw128(slot_addr(ks) + kk * 2048, Cfg::kChunk, 1024), id_pv,
+                     (any_pv[hh] || kk > 0) ? 1u : 0u);
+            };
+            if (ksteps == BK / 16) {
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)
-              // P of keys [16kk, 16kk+16): each column half of the head's S
-              // range holds its P at the start of that half
-              if (kk < ksteps)
-                mma_ts(tO(hh), tS(hh) + (kk / (BK / 32)) * (BK / 2) + (kk % (BK / 32)) * 8,
-                       desc_sw128(slot_addr(ks) + kk * 2048, Cfg::kChunk, 1024), id_pv,
-                       (any_pv[hh] || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < BK / 16; ++kk) pv_step(kk);
+            } else {
+              for (int kk = 0; kk < ksteps; ++kk) pv_step(kk);
+            }
             any_pv[hh] = true;
           }
           // this head's S (or P, read by the PV just issued, which runs

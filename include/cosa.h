@@ -162,6 +162,35 @@ COSA_API cosa_status cosa_decode_plan(const cosa_shape* shape, const void* q, co
                                       int32_t* hrm_count, float* block_score, uint8_t* hrm_flags,
                                       cudaStream_t stream);
 
+/* The attention of one decode step (shape->Nq == 1): OSK (technical summary
+ * Sec. 2.3) on the single query row of each head, at position Nkv - 1:
+ * visit order[b,h,0,0..count-1]; skip a visit when fp32(m_loc - m_run) < T,
+ * T = fp32(ln(skip_eps) * sqrt(d)) (with one row the tile-wide vote is the
+ * row's own test); fold the others into the softmax (scale 1/sqrt(d)).  The
+ * pages leave decoding to future work (Sec. 4): the decisions, skip bits and
+ * results are those of cosa_attend on the same one-row shape, computed by
+ * kernels shaped for a memory-bound step: the logits of every visited block
+ * in parallel, the decisions as a prefix-max scan (a skipped visit never
+ * raises the running max, since T <= 0), the P.V of the computed visits in
+ * parallel against their common maximum.  Logits are fp32 sums on the CUDA
+ * cores and P stays fp32, so on real-valued inputs a decision can differ
+ * from cosa_attend's where m_loc - m_run - T is within fp32 rounding of 0.
+ *  q          [B, Hq, 1, d] bf16.
+ *  order      [B, Hq, 1, kmax] int32 (cosa_decode_plan's); count [B, Hq, 1].
+ *  out        [B, Hq, 1, d] bf16 out; lse [B, Hq] fp32 out (nullable);
+ *             skip_bits [B, Hq, ceil(kmax/32)] uint32 out (nullable).
+ *  workspace  >= cosa_decode_attend_workspace_bytes(shape, kmax) bytes of
+ *             device memory, 256-byte aligned (logits of every visit, the
+ *             visits' row maxima, per-CTA partial sums).
+ * Entries of order outside [0, nKB) count as skipped visits.  Returns
+ * COSA_ESHAPE if Nq != 1, COSA_EWORKSPACE for a missing or small workspace,
+ * COSA_EUNSUPPORTED when kmax is too large for the scan's shared memory. */
+COSA_API size_t cosa_decode_attend_workspace_bytes(const cosa_shape* shape, int kmax);
+COSA_API cosa_status cosa_decode_attend(const cosa_shape* shape, const void* q, const void* k, const void* v,
+                                        const int32_t* page_table, const int32_t* order, const int32_t* count,
+                                        int kmax, double skip_eps, void* out, float* lse, uint32_t* skip_bits,
+                                        void* workspace, size_t ws_bytes, cudaStream_t stream);
+
 /* Block union ("CompactAttention: Accelerating Chunked Prefill with
  * Block-Union KV Selection", method, selection stage): turn a per-head
  * selection into one KV block table per (batch, kv-head group), the union

@@ -26,6 +26,10 @@ available here, so these synthetic inputs stand in for their shapes only):
   P_k = 2048 * 2^(k/2); their product peaks at lag 0 and decays over a few
   blocks.
 * V = z.
+* recipe "planned" (``Workload.recipe``), the first plan of the benchmark:
+  Q_DIR_PLANNED = 2 instead of 16, and needle blocks get
+  K += NEEDLE_SCALE * ubar_g (no sqrt(d) factor); sinks as above.  Attention
+  is then far less concentrated, and the in-kernel skip test fires less.
 * the integer grid variant draws Q, K, V uniformly from {-2,...,2}; every
   pooled value and every logit is then exact in bf16 / fp32.  With structure
   on, a per-kv-head integer direction w_g in {-1, 0, 1}^d (nonzero on dims
@@ -46,6 +50,7 @@ from typing import Optional
 import torch
 
 Q_DIR = 16.0
+Q_DIR_PLANNED = 2.0
 MU_STD = 0.5
 SINK_SCALE = 3.0
 NEEDLE_SCALE = 3.0
@@ -77,6 +82,7 @@ class Workload:
     local_window: bool = False
     budgets: tuple = (0.1,)
     eps: float = 1e-4
+    recipe: str = "default"  # "default" or "planned" (weaker query direction and needles, see above)
 
     @property
     def n_qblocks(self) -> int:
@@ -196,7 +202,7 @@ def generate(wl: Workload, grid: bool = False, rank: int = 0) -> Inputs:
             for h in range(Hq):
                 x = torch.randn(Nq, d, generator=gq)
                 if wl.structured:
-                    x += Q_DIR * u[b, h]
+                    x += (Q_DIR_PLANNED if wl.recipe == "planned" else Q_DIR) * u[b, h]
                     if loc_q is not None:
                         x += loc_q
                 q[b, h] = x.to(torch.bfloat16)
@@ -209,7 +215,8 @@ def generate(wl: Workload, grid: bool = False, rank: int = 0) -> Inputs:
                     if wl.n_needle > 0 and n_blk > 1:
                         picks = torch.randperm(n_blk - 1, generator=gn)[: wl.n_needle] + 1
                         for blk in picks.tolist():
-                            x[blk * 128:(blk + 1) * 128] += NEEDLE_SCALE * sq * ubar[b, g]
+                            x[blk * 128:(blk + 1) * 128] += \
+                                NEEDLE_SCALE * (1.0 if wl.recipe == "planned" else sq) * ubar[b, g]
                     if loc_k is not None:
                         x += loc_k
                 k[b, g] = x.to(torch.bfloat16)

@@ -76,3 +76,18 @@ def test_dense_causal_flops_closed_form():
         pairs = sum(min(wl.Nkv, wl.Nkv - wl.Nq + i + 1) for i in range(wl.Nq))
         assert wl.dense_causal_flops() == 4.0 * wl.B * wl.Hq * wl.d * pairs
         assert abs(wl.dense_causal_flops() / expect[name] - 1) < 5e-3, name
+
+
+def test_planned_recipe_weakens_the_structure():
+    """The "planned" recipe (query direction 2, needles 3 * ubar) draws the
+    same noise as the default one and differs only by the structure terms:
+    queries move by (16 - 2) * u_h, needle keys by 3 * (sqrt(d) - 1) * ubar_g."""
+    wl = _small(Nq=1024, Nkv=1024, bk=128)
+    a = synth.generate(wl)
+    b = synth.generate(wl.replace(recipe="planned"))
+    assert torch.equal(a.v, b.v)
+    dq = (a.q.float() - b.q.float()).norm(dim=-1)
+    assert abs(dq.mean().item() - 14.0) < 0.3          # |(16 - 2) u_h| = 14, up to bf16 rounding
+    dk = (a.k.float() - b.k.float()).norm(dim=-1)
+    assert dk[:, :, :4].abs().max().item() < 0.2       # sinks unchanged
+    assert abs(dk.max().item() - 3.0 * (128 ** 0.5 - 1.0)) < 0.5
