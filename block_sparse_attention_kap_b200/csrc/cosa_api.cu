@@ -421,6 +421,7 @@ cosa_status attend_impl(const cosa_shape* shape, const void* q, const void* k, c
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)s.d));
   p.out = static_cast<uint16_t*>(out); p.lse = lse; p.skip_bits = skip_bits; p.skip_words = cdiv(kmax, 32);
   p.status = dev_status;
+  p.kv_tail = s.Nkv % s.bk;
   p.wait_limit_ns = wait_limit_ns;
   p.stall_test = stall_test;
   if (group) return launch_status(launch_osk_group(tm_q, tm_k, tm_v, p, s.bk, stream));

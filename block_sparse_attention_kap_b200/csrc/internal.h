@@ -91,6 +91,7 @@ struct OskParams {
   uint32_t* skip_bits;          // optional [B, Hq, nQB, skip_words]
   int skip_words;
   uint32_t* status;
+  int kv_tail;                  // keys in the last KV block when it is ragged (Nkv % bk), else 0
   uint64_t wait_limit_ns;       // limit of every pipeline wait (1 s; shorter only in the test hook)
   int stall_test;               // 0; 1 only in the wait-timeout test hook
 };

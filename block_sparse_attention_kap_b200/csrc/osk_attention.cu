@@ -194,8 +194,8 @@ osk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           if (!wait_slot(ks)) break;
           // a ragged last block: no MMA step past the end of the cache, and the
           // non-key rows of the last step zeroed (see clear_v_tail)
-          const int valid = (jv >= 0 && jv < p.nkb) ? min(BK, p.Nkv - jv * BK) : BK;   // >= 1
-          const int ksteps = clear_v_tail(slot(ks), Cfg::kChunk, valid);
+          int ksteps = BK / 16;
+          if (p.kv_tail && jv == p.nkb - 1) ksteps = clear_v_tail(slot(ks), Cfg::kChunk, p.kv_tail);
           tc_fence_after();
           // P of keys [16kk, 16kk+16): each column half packs its P at the
           // start of its own S range (TMEM columns half*BK/2 + ...)

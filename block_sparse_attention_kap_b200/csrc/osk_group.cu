@@ -200,8 +200,7 @@ osk_group_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
               if (!wait_slot(ks)) { ok = false; break; }
               // a ragged last block: no MMA step past the end of the cache,
               // and the non-key rows of the last step zeroed (clear_v_tail)
-              const int valid = (jv >= 0 && jv < p.nkb) ? min(BK, p.Nkv - jv * BK) : BK;   // >= 1
-              ksteps = clear_v_tail(slot(ks), Cfg::kChunk, valid);
+              if (p.kv_tail && jv == p.nkb - 1) ksteps = clear_v_tail(slot(ks), Cfg::kChunk, p.kv_tail);
               v_seen = true;
             }
             tc_fence_after();
