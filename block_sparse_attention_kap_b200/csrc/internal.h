@@ -48,6 +48,7 @@ struct ScoreParams {
   int kpb;                      // pooled keys per KV block (bk / s)
   int n_row_tiles;              // ceil(nqp / 128)
   int splits;                   // S: each row tile's key tiles are cut into S work items
+  int rpq;                      // pooled rows per Q-block (bq / s): the Bs layout groups them
   float* bs;                    // [B*Hq, n_row_tiles, nKB, 128] max-pooled block scores
   float* part_max;              // [B*Hq, n_row_tiles, S, 2, 128] row max of each item and column half
   int32_t* part_arg;            // ... and the first block attaining it (-1: none)

@@ -60,13 +60,13 @@ __device__ __forceinline__ void rank_qblock(const SortParams& p, int row, int pk
   }
 
   // ------------------------------------------------------------ MaxNorm, aggregate, HRM -> ranking keys
-  const float* bs = p.bs + ((size_t)hb * p.n_row_tiles + R) * p.nkb * kTileRows + row0;
+  const float* bs = p.bs + ((size_t)hb * p.n_row_tiles + R) * p.nkb * kTileRows + (size_t)(row0 / RPQ) * p.nkb * RPQ;
   const size_t out_row = (size_t)row * p.nkb;
   const uint32_t hrm_key = orderable(1.0f);
   int hrm = 0;
   for (int j = lane; j < n; j += 32) {
     float v[RPQ];
-    const float* src = bs + (size_t)j * kTileRows;
+    const float* src = bs + (size_t)j * RPQ;
     if constexpr (RPQ % 4 == 0) {
 #pragma unroll
       for (int i = 0; i < RPQ; i += 4) {

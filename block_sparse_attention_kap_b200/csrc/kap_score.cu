@@ -169,8 +169,9 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
     const int climit = p.off_p + r;
     float rowmax = -INFINITY;
     int argj = -1;
-    // this row's Bs, [nKB][128 rows] per (head, row tile): coalesced across the warp
-    float* bs_row = p.bs + ((size_t)hb * p.n_row_tiles + R) * p.nkb * kTileRows + row;
+    // this row's Bs: per (head, row tile) [Q-block][nKB][rows of the Q-block],
+    // so kap_sort reads each Q-block's scores contiguously
+    float* bs_row = p.bs + ((size_t)hb * p.n_row_tiles + R) * p.nkb * kTileRows + (size_t)(row / p.rpq) * p.nkb * p.rpq + row % p.rpq;
     for (int u = 0; u < U; ++u) {
       const int st = u & 1;
       const int T = t0 + u;
@@ -208,7 +209,7 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
       const int j0 = T * BPT + half * BPH;                     // first block of this half
 #pragma unroll
       for (int jh = 0; jh < BPH; ++jh)
-        if (j0 + jh < p.nkb) bs_row[(size_t)(j0 + jh) * kTileRows] = bsv[jh];
+        if (j0 + jh < p.nkb) bs_row[(size_t)(j0 + jh) * p.rpq] = bsv[jh];
 #pragma unroll
       for (int jh = 0; jh < BPH; ++jh)
         if (bsv[jh] > rowmax) { rowmax = bsv[jh]; argj = j0 + jh; }
