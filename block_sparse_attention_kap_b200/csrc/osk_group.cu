@@ -68,13 +68,15 @@ osk_group_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   if (__syncthreads_or(failed)) return;
 
   const int tid = threadIdx.x, warp = tid >> 5;
-  // heaviest (last) Q-blocks first; the head pairs of a kv-head adjacent
+  // one kv-head (and batch) at a time, heaviest (last) Q-blocks first, the
+  // head pairs of the kv-head adjacent (as in osk_attention: the K/V tiles of
+  // the resident CTAs stay in L2)
   const int pairs = p.G / kHeads;
   int x = blockIdx.x;
   const int pr = x % pairs; x /= pairs;
+  const int I = p.nqb - 1 - x % p.nqb; x /= p.nqb;
   const int g = x % p.Hkv; x /= p.Hkv;
-  const int b = x % p.B; x /= p.B;
-  const int I = p.nqb - 1 - x;
+  const int b = x;
   const int h0 = g * p.G + kHeads * pr;
   const size_t orow = ((size_t)(b * p.Hkv + g)) * p.nqb + I;  // the group's order row
   const int32_t* ord = p.order + orow * p.kmax;
