@@ -51,7 +51,7 @@ def parse():
                     help="override the workload's query/kv head counts (a smaller case of the same layer, "
                          "e.g. for profiling); the workload is then reported as NAME[hqHQ:hkvHKV]")
     ap.add_argument("--recipe", default="default", choices=["default", "planned"],
-                    help="input recipe: the default one, or the first plan's weaker structure")
+                    help="input recipe: the default one, or a weaker structure (query direction 2, needles without sqrt(d))")
     ap.add_argument("--budget", type=float, default=None)
     ap.add_argument("--eps", type=float, default=None)
     ap.add_argument("--impl", default="cosa", choices=["cosa", "reference"])

@@ -26,8 +26,8 @@ available here, so these synthetic inputs stand in for their shapes only):
   P_k = 2048 * 2^(k/2); their product peaks at lag 0 and decays over a few
   blocks.
 * V = z.
-* recipe "planned" (``Workload.recipe``), the first plan of the benchmark:
-  Q_DIR_PLANNED = 2 instead of 16, and needle blocks get
+* recipe "planned" (``Workload.recipe``), a weaker structure drawn from the
+  same noise: Q_DIR_PLANNED = 2 instead of 16, and needle blocks get
   K += NEEDLE_SCALE * ubar_g (no sqrt(d) factor); sinks as above.  Attention
   is then far less concentrated, and the in-kernel skip test fires less.
 * the integer grid variant draws Q, K, V uniformly from {-2,...,2}; every
