@@ -1,9 +1,8 @@
 // kap_sort: the ranking and flag-grouped sorting of the Kernel-Aware Proxy
 // (CoSA technical summary Sec. 2.2) as a kernel of its own: one warp per
 // (b, h, Q-block), several per CTA, synchronised only with __syncwarp; the
-// work of each warp is rank_qblock (kap_rank.cuh).  kap_score runs the same
-// ranking in the last work item of each row tile whenever the per-warp
-// scratch fits its shared memory; this kernel serves the other shapes.
+// work of each warp is rank_qblock (kap_rank.cuh).  It runs after kap_score,
+// whose block scores Bs and partial row maxima it reads.
 #include "kap_rank.cuh"
 
 namespace cosa {
