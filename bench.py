@@ -717,6 +717,33 @@ def main():
     assert m.device_status() == 0
     assert torch.equal(outs_h[(esteps - 1) % 2], outs[(esteps - 1) % 2].cpu())
 
+    # the same copies in the same pattern with no compute between them: the
+    # host link's floor for this step's bytes
+    def copies_only(nsteps):
+        for i in range(nsteps):
+            bi = i % 2
+            qd, kd, vd, ptd = dev_in[bi]
+            with torch.cuda.stream(s_h2d):
+                qd.copy_(host[0], non_blocking=True)
+                kd.copy_(host[1], non_blocking=True)
+                vd.copy_(host[2], non_blocking=True)
+                if ptd is not None:
+                    ptd.copy_(pt_h, non_blocking=True)
+            with torch.cuda.stream(s_d2h):
+                outs_h[bi].copy_(outs[bi], non_blocking=True)
+
+    torch.cuda.synchronize()
+    a, b = ev(), ev()
+    a.record(stream)
+    s_h2d.wait_stream(stream)
+    s_d2h.wait_stream(stream)
+    copies_only(esteps)
+    stream.wait_stream(s_d2h)
+    stream.wait_stream(s_h2d)
+    b.record(stream)
+    torch.cuda.synchronize()
+    copy_floor_ms = max_over_ranks([a.elapsed_time(b) / esteps], dist, dev)[0]
+
     # ---------------------------------------------------------- CPU baseline (rank 0, N = 1)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -743,7 +770,9 @@ def main():
             "cpu_baseline": cpu,
             "e2e": {"value": whole_job_tflops(dense_flops, world, e2e_ms), "unit": "TFLOP/s",
                     "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "steps": esteps, "pipelined": "copies in/out overlap the neighbouring steps' compute"},
+                    "steps": esteps, "pipelined": "copies in/out overlap the neighbouring steps' compute",
+                    "copy_floor_ms": copy_floor_ms,
+                    "copy_floor": "the same host-to-device and device-to-host copies per step with no compute"},
             "gpu_launches": 4 * args.steps,
             "clocks": clocks,
             "kap_ms": kap_ms, "osk_ms": osk_ms,
