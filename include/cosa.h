@@ -152,8 +152,9 @@ COSA_API cosa_status cosa_plan_chunk(const cosa_shape* shape, const void* q, con
  *  order      [B, Hq, 1, kmax] int32 out (kmax >= k), padded -1; count,
  *             hrm_count [B, Hq] out; block_score [B, Hq, nKB] fp32 and
  *             hrm_flags [B, Hq, nKB] uint8 out (nullable).
- * The decode step's attention is cosa_attend on the same shape (Nq = 1):
- * with one valid row the tile-wide skip vote is that row's own test.
+ * The decode step's attention is cosa_decode_attend (or cosa_attend) on the
+ * same shape (Nq = 1): with one valid row the tile-wide skip vote is that
+ * row's own test.
  * Returns COSA_ESHAPE if Nq != 1, COSA_EINVAL for null pointers, a budget
  * outside (0, 1], kp arguments out of range or kmax < k. */
 COSA_API cosa_status cosa_decode_plan(const cosa_shape* shape, const void* q, const void* k,
@@ -279,9 +280,9 @@ COSA_API cosa_status cosa_attend_group(const cosa_shape* shape, const void* q, c
  * waits (again bounded) for the copies it started, TMEM is released and the
  * CTA exits; CTAs that start after the status is set exit at once.  The
  * call returns COSA_OK; the CTAs that ran write zeros to their rows of
- * `out`, the others leave them as they were; the context stays usable: a test calls it to check that a wait that runs out
- * ends in an error status rather than a hang or a fault.  Not for use in
- * production.
+ * `out`, the others leave them as they were; the context stays usable.  A
+ * test calls it to check that a wait that runs out ends in an error status
+ * rather than a hang or a fault.  Not for use in production.
  *  dev_status     required; should be 0 before the call.
  *  wait_limit_ns  in [1e3, 1e9].
  * Returns COSA_EINVAL for a null dev_status or a limit out of range, and
