@@ -68,6 +68,7 @@ _lib.cosa_decode_attend.argtypes = [_S, _P, _P, _P, _P, _P, _P, ctypes.c_int, ct
                                     ctypes.c_size_t, _P]
 _lib.cosa_attend_group.argtypes = [_S, _P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_double, _P, _P, _P, _P, _P]
 _lib.cosa_test_attend_wait_timeout.argtypes = [_S, _P, _P, _P, _P, _P, _P, ctypes.c_int, _P, _P, ctypes.c_uint64, _P]
+_lib.cosa_check_order.argtypes = [_S, _P, _P, ctypes.c_int, ctypes.POINTER(ctypes.c_int64)]
 _lib.cosa_skip_threshold.argtypes = [ctypes.c_double, ctypes.c_int]
 _lib.cosa_skip_threshold.restype = ctypes.c_float
 _lib.cosa_status_string.argtypes = [ctypes.c_int]
@@ -77,7 +78,7 @@ EXPORTS = ("cosa_num_qblocks", "cosa_num_kblocks", "cosa_kmax", "cosa_plan_works
            "cosa_dense_order", "cosa_attend", "cosa_skip_threshold", "cosa_status_string", "cosa_version",
            "cosa_plan_static", "cosa_plan_chunk", "cosa_block_union", "cosa_decode_plan",
            "cosa_test_attend_wait_timeout", "cosa_attend_group", "cosa_decode_attend",
-           "cosa_decode_attend_workspace_bytes")
+           "cosa_decode_attend_workspace_bytes", "cosa_check_order")
 DEV_TIMEOUT_TMA, DEV_TIMEOUT_MMA, DEV_TIMEOUT_PIPE = 0x100, 0x200, 0x300
 STATIC_SCRATCH_BYTES = 64 << 20
 
@@ -137,6 +138,31 @@ def cosa_status_string(status: int) -> str:
 
 def cosa_version() -> int:
     return _lib.cosa_version()
+
+
+def cosa_check_order(shape: cosa_shape, order, count, kmax: Optional[int] = None) -> int:
+    """Check a visit order on the host before cosa_attend: order [B, Hq, nQB,
+    kmax] and count [B, Hq, nQB] int32 (copied to host memory if they are on
+    the GPU).  Returns 0 when every count is in [0, kmax] and every visited
+    block is causally visible to its Q-block and appears once in its row;
+    otherwise raises CosaError naming the first bad row and entry."""
+    if order.dtype != torch.int32 or count.dtype != torch.int32:
+        raise ValueError("order and count must be int32")
+    km = order.shape[-1] if kmax is None else kmax
+    o = order.detach().to("cpu").contiguous()
+    c = count.detach().to("cpu").contiguous()
+    if o.numel() != c.numel() * km:
+        raise ValueError(f"order has {o.numel()} entries, count {c.numel()} rows of kmax {km}")
+    bad = ctypes.c_int64(0)
+    st = _lib.cosa_check_order(ctypes.byref(shape), ctypes.c_void_p(o.data_ptr()), ctypes.c_void_p(c.data_ptr()),
+                               km, ctypes.byref(bad))
+    if st == 1 and bad.value < 0:
+        raise CosaError(st, f"cosa_check_order: count {int(c.view(-1)[-1 - bad.value])} of row {-1 - bad.value}")
+    if st == 1:
+        raise CosaError(st, f"cosa_check_order: row {bad.value // km}, visit {bad.value % km} "
+                            f"(block {int(o.view(-1)[bad.value])})")
+    _check(st, "cosa_check_order")
+    return 0
 
 
 def cosa_plan(shape: cosa_shape, q, k, page_table, budget: float, kmax: int, order, count,
@@ -441,6 +467,12 @@ class CoSA:
 
     def device_status(self) -> int:
         return int(self.status.item())
+
+    def check_plan(self, order, count) -> None:
+        """cosa_check_order on this shape: raises CosaError at the first visit
+        a caller-edited order must not make (a block visited twice, one its
+        Q-block cannot see, a count outside [0, kmax])."""
+        cosa_check_order(self.shape, order, count)
 
 
 def shape_of_workload(wl) -> cosa_shape:

@@ -4,8 +4,10 @@
 // stream.
 #include <cudaTypedefs.h>
 #include <cmath>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "cosa.h"
 #include "internal.h"
@@ -276,6 +278,39 @@ cosa_status cosa_plan_chunk(const cosa_shape* shape, const void* q, const void* 
   return plan_impl(&s, q, k, page_table, static_cast<uint16_t*>(kp_cache), (long long)s.B * s.Hkv * kp_capacity,
                    kp_capacity, kp_valid, budget, kmax, order, count, hrm_count, block_score, hrm_flags,
                    static_cast<uint8_t*>(workspace), dev_status, stream);
+}
+
+cosa_status cosa_check_order(const cosa_shape* shape, const int32_t* order_host, const int32_t* count_host,
+                             int kmax, int64_t* first_bad) {
+  if (first_bad) *first_bad = 0;
+  cosa_status st = check_shape(shape);
+  if (st != COSA_OK) return st;
+  if (kmax < 1) return COSA_ESHAPE;
+  const int nqb = n_qblocks(shape), nkb = n_kblocks(shape);
+  const long long rows = (long long)shape->B * shape->Hq * nqb;
+  if (rows == 0) return COSA_OK;
+  if (!order_host || !count_host) return COSA_EINVAL;
+  std::vector<uint64_t> seen((size_t)(nkb + 63) / 64);
+  for (long long row = 0; row < rows; ++row) {
+    const int n = count_host[row];
+    if (n < 0 || n > kmax) {
+      if (first_bad) *first_bad = -1 - row;
+      return COSA_EINVAL;
+    }
+    const int n_vis = causal_blocks(shape, (int)(row % nqb));
+    std::fill(seen.begin(), seen.end(), 0ull);
+    const int32_t* ord = order_host + row * kmax;
+    for (int t = 0; t < n; ++t) {
+      const int j = ord[t];
+      const bool bad = j < 0 || j >= n_vis || ((seen[(size_t)j >> 6] >> (j & 63)) & 1ull);
+      if (bad) {
+        if (first_bad) *first_bad = row * kmax + t;
+        return COSA_EINVAL;
+      }
+      seen[(size_t)j >> 6] |= 1ull << (j & 63);
+    }
+  }
+  return COSA_OK;
 }
 
 cosa_status cosa_dense_order(const cosa_shape* shape, int kmax, int32_t* order, int32_t* count,

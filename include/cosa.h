@@ -224,6 +224,22 @@ COSA_API cosa_status cosa_block_union(const cosa_shape* shape, const int32_t* or
 COSA_API cosa_status cosa_dense_order(const cosa_shape* shape, int kmax, int32_t* order, int32_t* count,
                              cudaStream_t stream);
 
+/* Host-side check of a visit order before cosa_attend, for a caller that
+ * edits or builds `order` itself (the computation-order mask of Sec. 2.1:
+ * a block visited twice would be folded into the softmax twice, which no
+ * kernel can detect).  order_host [B, Hq, nQB, kmax] and count_host
+ * [B, Hq, nQB] are int32 in HOST memory (copy them back first); nothing is
+ * launched.  Every count must lie in [0, kmax]; every entry t < count of a
+ * row must be a KV block its Q-block can see causally (0 <= j < n_I, as in
+ * cosa_kmax), and no block may appear twice in a row.  cosa_plan's and
+ * cosa_dense_order's results always pass.
+ *  first_bad  (nullable) out: the flat index row * kmax + t of the first bad
+ *             entry, or -1 - row for a bad count; 0 when all is well.
+ * Returns COSA_OK, COSA_EINVAL at the first bad count or entry (or a null
+ * array), COSA_ESHAPE for an invalid shape or kmax < 1. */
+COSA_API cosa_status cosa_check_order(const cosa_shape* shape, const int32_t* order_host,
+                                      const int32_t* count_host, int kmax, int64_t* first_bad);
+
 /* OSK, stage 2 (Sec. 2.3): for each (b, h, Q-block I) visit only the KV
  * blocks order[b,h,I,0..count-1], in that order (mask-skipped blocks are
  * never touched); per visited block compute S = Q K^T exactly, and skip the

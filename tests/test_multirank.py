@@ -32,7 +32,7 @@ def _worker(rank, world, port, out):
 
 def test_max_over_ranks_two_gloo_ranks():
     world = 2
-    manager = mp.Manager()
+    manager = mp.get_context("spawn").Manager()      # no fork of this multi-threaded process
     out = manager.dict()
     mp.start_processes(_worker, args=(world, _free_port(), out), nprocs=world, join=True, start_method="spawn")
     assert dict(out) == {0: [2.0, 10.0], 1: [2.0, 10.0]}
