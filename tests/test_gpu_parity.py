@@ -353,6 +353,25 @@ def _full_inputs(cosa, name, grid):
 # 2K single head at 25%, the 32K layer at 10%, the 128K layer at 10% and 5%,
 # the 4096-query chunk after a 128K paged cache at 10%, and the B=2 x 64K
 # sweep at 100% (threshold 0: must equal dense attention), 50, 20, 10, 5, 2%
+def check_plan_structure(cosa, m, plan, wl, budget):
+    """Every row of a full-size plan, not only the sampled ones: a visit order
+    cosa_attend may be given (cosa_check_order: causally visible blocks, none
+    twice), of exactly k_I = max(1, ceil(n_I * budget)) blocks (the budget
+    rule of cosa_kmax), padded with -1 past the count."""
+    cosa.cosa_check_order(m.shape, plan["order"], plan["count"])
+    nqb, nkb = wl.n_qblocks, cosa.cosa_num_kblocks(m.shape)
+    last = torch.clamp((torch.arange(nqb) + 1) * wl.bq, max=wl.Nq) - 1
+    n = torch.clamp((wl.Nkv - wl.Nq + last) // wl.bk + 1, max=nkb)
+    bp = round(budget * 10000)
+    k = torch.minimum(torch.clamp((n * bp + 9999) // 10000, min=1), n).to(torch.int32)
+    cnt = plan["count"].cpu().view(-1, nqb)
+    assert torch.equal(cnt, k.expand_as(cnt))
+    km = plan["order"].shape[-1]
+    o = plan["order"].cpu().view(-1, km)
+    past = torch.arange(km).view(1, -1) >= cnt.reshape(-1, 1)
+    assert bool((o[past] == -1).all())
+
+
 FULL_CASES = [("single_head_2k", 0.25, EPS), ("gqa_32k", 0.1, EPS), ("gqa_128k", 0.1, EPS), ("gqa_128k", 0.05, EPS),
               ("chunked_128k_paged", 0.1, EPS), ("sweep_64k_b2", 1.0, 0.0), ("sweep_64k_b2", 0.5, EPS),
               ("sweep_64k_b2", 0.2, EPS), ("sweep_64k_b2", 0.1, EPS), ("sweep_64k_b2", 0.05, EPS),
@@ -375,6 +394,7 @@ def test_full_size_sampled(cosa, name, budget, eps):
     plan = m.plan(dev[0], dev[1], budget, page_table=dev[3], scores=True)
     torch.cuda.synchronize()
     assert m.device_status() == 0
+    check_plan_structure(cosa, m, plan, wl, budget)
     sel = _samples(wl, 12, 3)
     idx = [(b * wl.Hq + h) * wl.n_qblocks + I for b, h, I in sel]
     km = plan["order"].shape[-1]
@@ -414,6 +434,7 @@ def test_full_size_grid_bit_exact(cosa, name, budget):
     plan = m.plan(dev[0], dev[1], budget, page_table=dev[3], scores=True)
     torch.cuda.synchronize()
     assert m.device_status() == 0
+    check_plan_structure(cosa, m, plan, wl, budget)
     n_rows = wl.B * wl.Hq * wl.n_qblocks
     sel = _samples(wl, 12, 5) if n_rows > 64 else None
     idx = [(b * wl.Hq + h) * wl.n_qblocks + I for b, h, I in sel] if sel else list(range(n_rows))
