@@ -372,6 +372,17 @@ def check_plan_structure(cosa, m, plan, wl, budget):
     assert bool((o[past] == -1).all())
 
 
+def check_attend_bounds(res, dev):
+    """Every row of a full-size attend: the output is a convex combination
+    of V rows (|out| <= max |v| up to the bf16 rounding of P and of out) and
+    finite, and the log-sum-exp is finite (every row sees at least one key
+    of the blocks it visits, the diagonal one among them)."""
+    out = res["out"].float()
+    assert bool(torch.isfinite(out).all())
+    assert float(out.abs().max()) <= float(dev[2].float().abs().max()) * (1 + 2.0 ** -7)
+    assert bool(torch.isfinite(res["lse"]).all())
+
+
 FULL_CASES = [("single_head_2k", 0.25, EPS), ("gqa_32k", 0.1, EPS), ("gqa_128k", 0.1, EPS), ("gqa_128k", 0.05, EPS),
               ("chunked_128k_paged", 0.1, EPS), ("sweep_64k_b2", 1.0, 0.0), ("sweep_64k_b2", 0.5, EPS),
               ("sweep_64k_b2", 0.2, EPS), ("sweep_64k_b2", 0.1, EPS), ("sweep_64k_b2", 0.05, EPS),
@@ -406,6 +417,7 @@ def test_full_size_sampled(cosa, name, budget, eps):
     order[idx] = ref["order"].cuda()
     count[idx] = ref["count"].cuda()
     res = gpu_attend(m, dev, order.view_as(plan["order"]), count.view_as(plan["count"]), eps)
+    check_attend_bounds(res, dev)
     o = oracle.osk(inp, ref["order"], ref["count"], eps, sel=sel)
     check_skips_and_out(cosa, res, o, wl, km, sel_idx=idx, eps=eps, literal=True)
     if budget == 1.0 and eps == 0.0:
