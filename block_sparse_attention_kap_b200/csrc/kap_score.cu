@@ -16,9 +16,11 @@
 // Q-block aggregate need every item of the row and run in kap_sort.
 // Every value is fp32; nothing is rounded after the contraction.
 //
-// Roles: warp 8 issues TMA and MMA; warps 0-7 are the epilogue, two per TMEM
-// lane quarter (row = 32*(warp%4) + lane), each taking one 64-column half of
-// every tile.
+// Roles: warp 8 (one thread) issues the MMAs, warp 9 (one thread) the TMA
+// loads, refilling a stage as soon as the MMAs of its tile have completed, so
+// the MMA issue never waits for a refill; warps 0-7 are the epilogue, two per
+// TMEM lane quarter (row = 32*(warp%4) + lane), each taking one 64-column
+// half of every tile.
 #include <cuda_bf16.h>
 #include "internal.h"
 #include "sm100.cuh"
@@ -28,8 +30,9 @@ namespace cosa {
 namespace {
 
 constexpr int kEpiWarps = 8;
-constexpr int kThreads = 32 * (kEpiWarps + 1);
-constexpr int kCtrl = 32 * kEpiWarps;            // the control thread
+constexpr int kThreads = 32 * (kEpiWarps + 2);
+constexpr int kCtrl = 32 * kEpiWarps;            // the MMA-issuing thread
+constexpr int kProd = 32 * (kEpiWarps + 1);      // the TMA-issuing thread
 constexpr uint32_t kTileBytes = 128 * 256;       // 128 rows x 128 bf16
 
 struct __align__(8) ScoreSmem {
@@ -102,8 +105,8 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
   tc_fence_after();
   const uint32_t tmem = sm->tmem_base;
 
-  if (tid == kCtrl) {
-    // ------------------------------------------------ control: TMA + MMA issue
+  if (tid == kProd) {
+    // ------------------------------------------------ producer: TMA loads
     tma_prefetch_desc(&tm_qp);
     tma_prefetch_desc(&tm_kp);
     const int qp_y = (b * p.Hq + h) * p.nqp + r_first;
@@ -113,16 +116,29 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
       tma_load_2d(sQ, &tm_qp, &sm->q_full, 0, qp_y);
       tma_load_2d(sQ + 16384, &tm_qp, &sm->q_full, 64, qp_y);
     }
-    uint32_t busy = 0u;    // stage bits: a key-tile load issued and not yet seen complete
-    uint32_t kph = 0u;     // stage bits: parity of the next completion on that stage
-    for (int u = 0; u < 2 && u < U; ++u) {
-      uint8_t* dst = sK + u * kTileBytes;
+    int loads[2] = {0, 0};   // key-tile loads issued on each stage
+    auto load = [&](int st, int u) {
+      uint8_t* dst = sK + st * kTileBytes;
       const int y = kp_y0 + (t0 + u) * kTileRows;
-      busy |= 1u << u;
-      mbar_arrive_expect_tx(&sm->k_full[u], kTileBytes);
-      tma_load_2d(dst, &tm_kp, &sm->k_full[u], 0, y);
-      tma_load_2d(dst + 16384, &tm_kp, &sm->k_full[u], 64, y);
+      ++loads[st];
+      mbar_arrive_expect_tx(&sm->k_full[st], kTileBytes);
+      tma_load_2d(dst, &tm_kp, &sm->k_full[st], 0, y);
+      tma_load_2d(dst + 16384, &tm_kp, &sm->k_full[st], 64, y);
+    };
+    for (int u = 0; u < 2 && u < U; ++u) load(u, u);
+    // refill a stage with tile u + 2 once the MMAs of tile u have completed
+    for (int u = 0; u + 2 < U; ++u) {
+      if (!wait_or_abort(&sm->s_full[u & 1], (u >> 1) & 1, abort, p.status, DEV_TIMEOUT_MMA)) break;
+      load(u & 1, u + 2);
     }
+    // no copy may still be writing shared memory when the CTA exits: wait
+    // (bounded) for the last load of each stage and for Q; on the normal path
+    // the issuing thread has seen them all complete already
+    if (U > 0) mbar_wait(&sm->q_full, 0);
+    for (int st = 0; st < 2; ++st)
+      if (loads[st] > 0) mbar_wait(&sm->k_full[st], (uint32_t)(loads[st] - 1) & 1u);
+  } else if (tid == kCtrl) {
+    // ------------------------------------------------ MMA issue
     const bool q_seen = U > 0 && wait_or_abort(&sm->q_full, 0, abort, p.status, DEV_TIMEOUT_TMA);
     bool ok = q_seen;
     const uint32_t idesc = idesc_bf16(128, 128, false, false);
@@ -131,8 +147,6 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
       const int st = u & 1;
       const uint32_t ph = (u >> 1) & 1;
       if (!wait_or_abort(&sm->k_full[st], ph, abort, p.status, DEV_TIMEOUT_TMA)) break;
-      busy &= ~(1u << st);
-      kph ^= 1u << st;
       if (u >= 2 && !wait_or_abort(&sm->s_free[st], ((u >> 1) - 1) & 1, abort, p.status, DEV_TIMEOUT_PIPE)) break;
       tc_fence_after();
       const uint32_t k_addr = smem_u32(sK + st * kTileBytes);
@@ -140,26 +154,10 @@ kap_score_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constan
       for (int kk = 0; kk < 8; ++kk)
         mma_ss(tmem + st * 128, tile_desc(q_addr, kk), tile_desc(k_addr, kk), idesc, kk > 0);
       tc_commit(&sm->s_full[st]);
-      if (u + 2 < U) {
-        // refill this stage once the MMA that reads it has completed
-        if (!wait_or_abort(&sm->s_full[st], ph, abort, p.status, DEV_TIMEOUT_MMA)) break;
-        uint8_t* dst = sK + st * kTileBytes;
-        const int y = kp_y0 + (t0 + u + 2) * kTileRows;
-        busy |= 1u << st;
-        mbar_arrive_expect_tx(&sm->k_full[st], kTileBytes);
-        tma_load_2d(dst, &tm_kp, &sm->k_full[st], 0, y);
-        tma_load_2d(dst + 16384, &tm_kp, &sm->k_full[st], 64, y);
-      }
     }
     // every MMA this thread issued has completed before TMEM is released
     tc_commit(&sm->drained);
     mbar_wait(&sm->drained, 0);
-    // no copy may still be writing shared memory when the CTA exits: after a
-    // failed wait, wait again (bounded) for the loads not yet seen complete
-    // (one per stage at most; none on the normal path)
-    if (U > 0 && !q_seen) mbar_wait(&sm->q_full, 0);
-    for (int st = 0; st < 2; ++st)
-      if (busy & (1u << st)) mbar_wait(&sm->k_full[st], (kph >> st) & 1u);
   } else if (warp < kEpiWarps) {
     // ------------------------------------------------ epilogue: one pooled row, one column half
     const int quarter = warp & 3, half = warp >> 2;
