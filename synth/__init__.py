@@ -7,7 +7,7 @@ paged KV cache).  It holds none of the method's arithmetic: no pooling, no
 scores, no softmax.  Both the CPU oracle (``oracle/``) and the CUDA path
 (``block_sparse_attention_kap_b200``) consume what it returns.
 
-Recipe (every constant below is a choice of this build; the pages give no
+Recipe (every constant below is a choice made here; the pages give no
 data distribution, they measure on RULER / LongBench-v2, which are not
 available here, so these synthetic inputs stand in for their shapes only):
 
